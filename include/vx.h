@@ -1,0 +1,196 @@
+/*
+ * vx.h -- C ABI of libvx: block top-k sparse attention decode over a paged KV cache,
+ * hand-written CUDA for B200 (sm_100a).
+ *
+ * The method (Vortex: Efficient and Programmable Sparse Attention Serving for AI Agents,
+ * paper note, section 系统设计 1 "vFlow", the block top-k example): a cache stage keeps
+ * one key centroid per KV page; an indexer scores every page by the product of the query
+ * with the centroids, keeps the top-k pages, and exact softmax attention runs on those
+ * pages only.  The paged layout (batch size, pointer array, page index structure) is the
+ * one of section 系统设计 2 "vTensor"; top-k is the radix top-k of section 系统设计 3
+ * with an optional stochastic-early-termination mode.
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * Pointers named *_cache, q, centroids, scores, sel, out, lse, ws, err and every array
+ * of vx_page_table are DEVICE pointers; vx_geometry and vx_page_table themselves are
+ * read on the host during the call and may be freed when it returns.  `stream` is a
+ * cudaStream_t (NULL = the legacy default stream).
+ *
+ * Ownership: the caller allocates and owns every buffer and keeps it alive until the
+ * stream has passed the call.  The library allocates no device memory and keeps no
+ * device state; calls are asynchronous and stream-ordered and never synchronise the
+ * host.  Calls on different streams may run concurrently when they write disjoint
+ * buffers (outputs, workspace, err).
+ *
+ * Layouts (row-major, element types in brackets):
+ *   k_cache    [num_pool_pages][num_kv_heads][page_size][head_dim_qk]  (bf16)
+ *   v_cache    [num_pool_pages][num_kv_heads][page_size][head_dim_v]   (bf16); ignored
+ *              when mla_shared_kv = 1: the value of a token is then the first head_dim_v
+ *              dims of its key row (MLA latent).
+ *   centroids  [num_pool_pages][num_kv_heads][head_dim_qk]             (bf16), keyed by
+ *              physical page so a centroid moves with its page.
+ *   q          [batch][num_q_heads][head_dim_qk]                       (bf16)
+ *   scores     [batch][num_kv_heads][max_pages]                        (fp32)
+ *   sel        [batch][num_kv_heads][k]  logical page indices          (int32), ascending,
+ *              -1 in the slots past k_eff = min(k, n_b)
+ *   out        [batch][num_q_heads][head_dim_v]                        (bf16)
+ *   lse        [batch][num_q_heads]  natural-log sum of exp(logits)    (fp32)
+ * Query head g belongs to KV head g / (num_q_heads / num_kv_heads) (GQA grouping).
+ * Request b holds seq_lens[b] tokens in n_b = ceil(seq_lens[b] / page_size) logical
+ * pages; logical page j is physical page page_indices[page_ptr[b] + j]; token t of the
+ * request sits in slot t % page_size of logical page t / page_size.  Slots past the
+ * length are never read into a result, whatever they hold.
+ * Every device pointer must be 16-byte aligned.
+ *
+ * Errors: argument problems are found on the host before anything is launched and
+ * returned as VX_ERR_INVALID_ARG / VX_ERR_UNSUPPORTED / VX_ERR_WORKSPACE; a failed
+ * launch returns VX_ERR_CUDA.  vx_last_error() then holds a message (per host thread).
+ * Problems in device data (a page id outside the pool, a length out of range, a
+ * selected page outside the request) are found by the kernels, which skip the bad item
+ * and OR a VX_DATA_* bit into *err (a device int32; may be NULL).  Kernels never trap
+ * and never wait without a time limit; a wait that runs out sets VX_DATA_TIMEOUT.
+ */
+#ifndef VX_H
+#define VX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VX_OK = 0,
+    VX_ERR_INVALID_ARG = 1, /* NULL or misaligned pointer, bad size, inconsistent geometry */
+    VX_ERR_UNSUPPORTED = 2, /* well-formed but not built: head dims, page size, group size */
+    VX_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than vx_workspace_size() */
+    VX_ERR_CUDA = 4         /* a CUDA runtime call or kernel launch failed */
+} vx_status;
+
+/* bits OR-ed into *err by the kernels */
+#define VX_DATA_BAD_PAGE_ID 1u   /* page_indices entry outside [0, num_pool_pages) */
+#define VX_DATA_BAD_SEQ_LEN 2u   /* seq_lens[b] < 1 or > max_pages * page_size */
+#define VX_DATA_BAD_SELECTION 4u /* sel entry >= n_b (entries < 0 are empty slots) */
+#define VX_DATA_TIMEOUT 8u       /* a bounded wait inside a kernel ran out */
+
+typedef struct {
+    int32_t batch;         /* B >= 1 */
+    int32_t num_q_heads;   /* Hq, a multiple of num_kv_heads */
+    int32_t num_kv_heads;  /* Hkv */
+    int32_t head_dim_qk;   /* key / score dim: 64 or 128 (GQA), 576 (MLA latent+rope) */
+    int32_t head_dim_v;    /* value dim: = head_dim_qk (GQA), 512 (MLA) */
+    int32_t page_size;     /* P tokens per page: 16, 32 or 64 (MLA: 64) */
+    int32_t mla_shared_kv; /* 1: V = first head_dim_v dims of the K row; v_cache unused */
+    int64_t num_pool_pages;
+} vx_geometry;
+
+typedef struct {
+    const int32_t *page_ptr;     /* [B] start of request b's row in page_indices */
+    const int32_t *page_indices; /* physical page ids, row b holds n_b entries */
+    const int32_t *seq_lens;     /* [B] valid tokens, 1 <= seq_lens[b] <= max_pages * P */
+    int32_t max_pages;           /* host bound on n_b over the batch; sizes scores rows */
+} vx_page_table;
+
+/*
+ * Cache stage: key centroid of a page = mean of the keys of its valid tokens, per KV
+ * head, stored as bf16 (the cache's element type) after one round-to-nearest-even of
+ * the fp32 mean (paper note, 系统设计 1: the cache stage keeps a per-block key centroid
+ * that does not depend on the query).
+ *   k_new == NULL: rebuild.  Recompute the centroid of every page of every request
+ *       holding a position >= first_pos[b] (first_pos NULL: every page).  Use after a
+ *       prefill or a bulk load.  v_cache, v_new unused.
+ *   k_new != NULL: append one decode token per request.  seq_lens already counts the
+ *       new token and its page is installed in the table; the token (k_new [B][Hkv][Dqk],
+ *       v_new [B][Hkv][Dv], v_new ignored for MLA) is written into slot
+ *       (seq_lens[b]-1) % P of its page and that page's centroid is recomputed from its
+ *       keys.  first_pos unused.
+ * Writes: centroids (and, when appending, one slot of k_cache / v_cache per request).
+ */
+vx_status vx_centroid_update(const vx_geometry *geo, const vx_page_table *table, void *k_cache,
+                             void *v_cache, void *centroids, const void *k_new, const void *v_new,
+                             const int32_t *first_pos, int32_t *err, void *stream);
+
+/*
+ * Indexer: scores[b][h][j] = sum over the query heads g of KV group h of
+ * q[b][g][:score_dims] . centroid(page j of b, head h)[:score_dims], fp32, no softmax
+ * scale (paper note, 系统设计 1: blocks are scored by a matrix product of query and
+ * centroids; MLA experiment section: the rope-aware variant scores on all 576 latent +
+ * rope dims, the rope-unaware one on the 512 latent dims only).
+ * score_dims: 0 = head_dim_qk; else 1..head_dim_qk, a multiple of 8.
+ * Writes scores[b][h][j] for j < n_b only.
+ */
+vx_status vx_score_pages(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                         const void *centroids, int32_t score_dims, float *scores, int32_t *err,
+                         void *stream);
+
+/*
+ * Top-k pages per (request, KV head) row of scores (paper note, 系统设计 3: radix top-k,
+ * with stochastic early termination and remapping as the faster approximate option).
+ *   mode 0 (exact): the k_eff = min(k, n_b) pages of largest score; ties at the boundary
+ *       go to the lower page index; -0.0 ties with +0.0.  Radix select on order-
+ *       preserving 32-bit keys, most significant digit first.
+ *   mode 1 (approximate): remap each score to a 12-bit code
+ *       min(4095, floor((s - lo) * (4096 / (hi - lo)))) in fp32 (lo, hi: the row's min
+ *       and max; hi == lo gives 0); one histogram; every page above the boundary code b*
+ *       is taken and the slots left are filled from code b* in cyclic page order from
+ *       offset SplitMix64(seed) draw number (b * Hkv + h) mod n_b, with no refinement.
+ * Writes sel [B][Hkv][k]: chosen pages in ascending order, then -1.  k >= 1.
+ * Scores must be finite; NaN scores give an unspecified (but in-range) selection.
+ */
+vx_status vx_topk_pages(const vx_geometry *geo, const vx_page_table *table, const float *scores,
+                        int32_t k, int32_t mode, uint64_t seed, int32_t *sel, int32_t *err,
+                        void *stream);
+
+/*
+ * Exact softmax attention over the selected pages only (paper note, 系统设计 1: exact
+ * attention on the chosen blocks; 系统设计 3: the MLA geometry kernel), gathered through
+ * the page table.  For query head g of KV head h:
+ *   out = sum_t softmax_t(sm_scale * q . K_t) V_t,  lse = log sum_t exp(sm_scale q . K_t)
+ * over the valid tokens of the pages in sel[b][h] (entries < 0 skipped; entries must be
+ * distinct).  Split-K: the selected tokens are cut into num_splits contiguous chunks
+ * whose partial (o, max, sum) are merged with the log-sum-exp rule.
+ *   sm_scale <= 0 means 1 / sqrt(head_dim_qk).  num_splits 0 = planned from the SM count.
+ *   lse may be NULL.  A request with no attended token gets out = 0, lse = -inf.
+ * ws: device workspace of at least vx_workspace_size(geo, max_pages, k, num_splits)
+ * bytes (the split partials).
+ */
+vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                           const void *k_cache, const void *v_cache, const int32_t *sel, int32_t k,
+                           float sm_scale, int32_t num_splits, void *out, float *lse, void *ws,
+                           size_t ws_bytes, int32_t *err, void *stream);
+
+/*
+ * One whole decode step: vx_score_pages -> vx_topk_pages -> vx_sparse_decode, chained
+ * on `stream` with programmatic dependent launch so each kernel's start overlaps the
+ * previous one's tail (paper note, 系统设计 3: fusion of the sequence-local steps and
+ * workload planning).  Same arguments and results as the three calls.  scores_out and
+ * sel_out (may be NULL) receive the intermediate scores and selection; when NULL they
+ * live in the workspace.  score_dims as in vx_score_pages.
+ */
+vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                               const void *k_cache, const void *v_cache, const void *centroids,
+                               int32_t k, int32_t mode, uint64_t seed, float sm_scale,
+                               int32_t score_dims, int32_t num_splits, void *out, float *lse,
+                               float *scores_out, int32_t *sel_out, void *ws, size_t ws_bytes,
+                               int32_t *err, void *stream);
+
+/*
+ * Workspace bytes that vx_sparse_decode and vx_block_topk_decode need for this geometry,
+ * row bound, k and split count (0 = the planned count); 0 when the arguments are
+ * invalid (see vx_last_error).  Deterministic: the same inputs give the same size.
+ */
+size_t vx_workspace_size(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits);
+
+/* Split count num_splits = 0 resolves to on the current device for this geometry. */
+int32_t vx_planned_splits(const vx_geometry *geo, int32_t max_pages, int32_t k);
+
+const char *vx_status_string(vx_status s);
+const char *vx_last_error(void); /* message of the last failed call on this host thread */
+const char *vx_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VX_H */

@@ -1,0 +1,429 @@
+// k_decode.cu -- exact softmax attention over the selected pages (GQA) + split merge.
+//
+// Vortex paper note, section 系统设计 1: after the indexer keeps the top-k blocks, exact
+// softmax attention runs on those blocks only, gathered through the page table
+// (section 系统设计 2).  Section 系统设计 3's workload planning is the split of that
+// work into equal chunks sized from the SM count.
+//
+// Work decomposition.  Every (request, KV head) row owns k selection slots; each slot
+// is a page of P tokens = P/16 tiles of 16 tokens.  The rows' tiles form one flat list
+// of T = rows * k * P/16 units, cut into W contiguous chunks of equal length; one warp
+// processes one chunk (a persistent grid: W = SMs * warps per block by default).  A
+// warp's chunk may end inside one row and continue in the next: for every row it
+// touches it writes one partial (unnormalised o, running max, running sum) to the
+// workspace at slot (row + chunk), an index that is unique because chunks are
+// contiguous.  The merge kernel combines a row's partials with the log-sum-exp rule.
+// The result therefore depends only on the selection and W, never on where the pages
+// live in the pool.
+//
+// Per warp: a ring of DEC_STAGES stages in shared memory, each holding one K tile and
+// one V tile (16 tokens x D bf16 each), filled by TMA tensor loads (128-byte swizzle,
+// 64-column boxes) that complete on a per-stage mbarrier.  Unit metadata (selected
+// page, physical page, valid tokens) is resolved 32 units at a time, one per lane.
+// Per tile: S^T = K Q^T with mma.m16n8k16 (tokens x heads, heads padded to 8 per
+// n-tile), online softmax in base 2, P^T moved into the B-operand layout with
+// movmatrix, O^T += V^T P^T with ldmatrix.trans for V.  Value rows past the request's
+// length are zeroed in registers, so NaN in unused slots cannot leak.
+#include "vx_internal.h"
+
+namespace vx {
+
+struct TileMeta {
+    int32_t row;
+    int32_t nvalid;
+};
+
+struct Resolved {
+    int32_t row, z, y, nvalid;  // row, tensor-map page-head index, token offset, valid tokens
+    bool valid;
+};
+
+__device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u, int64_t u_end) {
+    Resolved rs{0, 0, 0, 0, false};
+    if (u >= u_end) return rs;
+    const int64_t r = u / a.units_per_row;
+    const int64_t rem = u - r * a.units_per_row;
+    const int i = static_cast<int>(rem / a.tiles_per_page);
+    const int sub = static_cast<int>(rem - (int64_t)i * a.tiles_per_page);
+    const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);
+    rs.row = static_cast<int32_t>(r);
+    const int32_t L = a.seq_lens[b];
+    if (L < 1 || L > a.max_pages * a.P) return rs;  // reported by the top-k kernel
+    const int32_t j = a.sel[r * a.k + i];
+    if (j < 0) return rs;
+    const int n = ceil_div(L, a.P);
+    if (j >= n) {
+        set_err(a.err, VX_DATA_BAD_SELECTION);
+        return rs;
+    }
+    const int tok0 = j * a.P + sub * DEC_TILE;
+    const int nvalid = min(DEC_TILE, L - tok0);
+    if (nvalid <= 0) return rs;
+    const int32_t phys = a.page_indices[a.page_ptr[b] + j];
+    if (phys < 0 || phys >= a.num_pool_pages) {
+        set_err(a.err, VX_DATA_BAD_PAGE_ID);
+        return rs;
+    }
+    rs.z = phys * a.Hkv + h;
+    rs.y = sub * DEC_TILE;
+    rs.nvalid = nvalid;
+    rs.valid = true;
+    return rs;
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(DEC_WARPS * 32, 1)
+    k_decode_gqa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const DecodeArgs a) {
+    constexpr int KB = D / 64;                      // 64-column TMA boxes per tile
+    constexpr int BOX_BYTES = DEC_TILE * 128;       // 16 rows x 128 bytes
+    constexpr int TILE_BYTES = KB * BOX_BYTES;      // 16 x D bf16
+    constexpr int STAGE_BYTES = 2 * TILE_BYTES;     // K tile + V tile
+    constexpr int MT = D / 16;                      // 16-dim steps
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;  // 128-byte swizzle wants 1 KB alignment
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g4 = lane >> 2, q4 = lane & 3;
+    const uint32_t stage0 = base + (uint32_t)(warp * DEC_STAGES) * STAGE_BYTES;
+    const uint32_t bar0 = base + (uint32_t)(DEC_WARPS * DEC_STAGES) * STAGE_BYTES + (uint32_t)(warp * DEC_STAGES) * 8u;
+    TileMeta *meta = reinterpret_cast<TileMeta *>(smem_raw + (base - raw) + DEC_WARPS * DEC_STAGES * STAGE_BYTES +
+                                                  DEC_WARPS * DEC_STAGES * 8) +
+                     warp * DEC_STAGES;
+
+    pdl_launch_dependents();
+    if (lane == 0) {
+        for (int s = 0; s < DEC_STAGES; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    __syncwarp();
+
+    const int64_t c = (int64_t)blockIdx.x * DEC_WARPS + warp;
+    if (c >= a.chunks) return;
+    const int64_t u_begin = chunk_start(c, a.units, a.chunks);
+    const int64_t u_end = chunk_start(c + 1, a.units, a.chunks);
+    const int64_t row_first = u_begin / a.units_per_row;
+    const int64_t row_last = (u_end - 1) / a.units_per_row;
+
+    pdl_wait();  // the selection comes from the previous kernel
+
+    // ---- per-row state
+    uint32_t qf[NT][MT][2];
+    float acc[NT][MT][4];
+    float m_run[NT][2], l_run[NT][2];
+    int64_t cur_row = -1;
+    int64_t flushed_to = row_first - 1;  // rows <= flushed_to have their partial written
+
+    auto write_empty = [&](int64_t r) {
+        if (lane < a.G) {
+            float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
+            ml[0] = -INFINITY;
+            ml[1] = 0.f;
+        }
+    };
+    auto flush = [&](int64_t r) {
+        float lt[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float v = l_run[nt][i];
+                v += __shfl_xor_sync(FULL, v, 4);
+                v += __shfl_xor_sync(FULL, v, 8);
+                v += __shfl_xor_sync(FULL, v, 16);
+                lt[nt][i] = v;
+            }
+        const int64_t slot = r + c;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int head = nt * 8 + 2 * q4 + (e & 1);
+                    const int dim = mt * 16 + g4 + 8 * (e >> 1);
+                    if (head < a.G) a.o_part[(slot * a.G + head) * a.Dv + dim] = acc[nt][mt][e];
+                }
+        if (g4 == 0) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int head = nt * 8 + 2 * q4 + i;
+                    if (head < a.G) {
+                        float *ml = a.ml_part + (slot * a.G + head) * 2;
+                        ml[0] = m_run[nt][i];
+                        ml[1] = lt[nt][i];
+                    }
+                }
+        }
+    };
+    auto start_row = [&](int64_t r) {
+        const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);
+        const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)h * a.G) * D;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = nt * 8 + g4;
+#pragma unroll
+            for (int kk = 0; kk < MT; ++kk) {
+                if (head < a.G) {
+                    const uint32_t *qp = reinterpret_cast<const uint32_t *>(qb + (size_t)head * D + kk * 16 + 2 * q4);
+                    qf[nt][kk][0] = qp[0];
+                    qf[nt][kk][1] = qp[4];  // +8 dims
+                } else {
+                    qf[nt][kk][0] = 0u;
+                    qf[nt][kk][1] = 0u;
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                m_run[nt][i] = -INFINITY;
+                l_run[nt][i] = 0.f;
+            }
+        }
+    };
+
+    // ---- pipeline
+    int64_t batch = u_begin;
+    Resolved rs = resolve_unit(a, batch + lane, u_end);
+    uint32_t pending = __ballot_sync(FULL, rs.valid);
+    uint32_t issued = 0, consumed = 0;
+    bool failed = false;
+
+    for (;;) {
+        // issue loads until the ring is full or the chunk is exhausted
+        while (issued - consumed < DEC_STAGES) {
+            if (pending == 0) {
+                batch += 32;
+                if (batch >= u_end) break;
+                rs = resolve_unit(a, batch + lane, u_end);
+                pending = __ballot_sync(FULL, rs.valid);
+                continue;
+            }
+            const int src = __ffs(pending) - 1;
+            pending &= pending - 1;
+            const int32_t row = __shfl_sync(FULL, rs.row, src);
+            const int32_t z = __shfl_sync(FULL, rs.z, src);
+            const int32_t y = __shfl_sync(FULL, rs.y, src);
+            const int32_t nv = __shfl_sync(FULL, rs.nvalid, src);
+            const int st = static_cast<int>(issued % DEC_STAGES);
+            if (lane == 0) {
+                meta[st].row = row;
+                meta[st].nvalid = nv;
+                const uint32_t bar = bar0 + 8u * st;
+                const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
+                fence_proxy_async_smem();  // earlier generic reads of this stage come first
+                mbar_arrive_expect_tx(bar, STAGE_BYTES);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_3d(sK + kb * BOX_BYTES, &tmK, kb * 64, y, z, bar);
+                    tma_load_3d(sK + TILE_BYTES + kb * BOX_BYTES, &tmV, kb * 64, y, z, bar);
+                }
+            }
+            __syncwarp();
+            ++issued;
+        }
+        if (consumed == issued) break;
+
+        const int st = static_cast<int>(consumed % DEC_STAGES);
+        const uint32_t bar = bar0 + 8u * st;
+        const bool ok = __all_sync(FULL, mbar_wait_bounded(bar, (consumed / DEC_STAGES) & 1u));
+        if (!ok) {
+            failed = true;
+            break;
+        }
+        const int64_t row = meta[st].row;
+        const int nvalid = meta[st].nvalid;
+        if (row != cur_row) {
+            if (cur_row >= 0) {
+                flush(cur_row);
+                flushed_to = cur_row;
+            }
+            for (int64_t r = flushed_to + 1; r < row; ++r) write_empty(r);
+            flushed_to = row - 1;
+            start_row(row);
+            cur_row = row;
+        }
+
+        const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
+        const uint32_t sV = sK + TILE_BYTES;
+
+        // S^T[token][head] = K . Q^T
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+        {
+            const int mi = lane >> 3, rr = lane & 7;
+            const int tok = rr + 8 * (mi & 1);
+#pragma unroll
+            for (int kk = 0; kk < MT; ++kk) {
+                const int chunk = (kk & 3) * 2 + (mi >> 1);
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(sK + (kk >> 2) * BOX_BYTES + swz128(tok, chunk), a0, a1, a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+            }
+        }
+        // online softmax (base 2), tokens >= nvalid masked
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float x[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = g4 + 8 * (e >> 1);
+                x[e] = tok < nvalid ? s[nt][e] * a.scale_log2 : -INFINITY;
+            }
+            float alpha[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float mx = fmaxf(x[i], x[i + 2]);
+                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+                const float m_new = fmaxf(m_run[nt][i], mx);
+                alpha[i] = exp2f(m_run[nt][i] - m_new);
+                m_run[nt][i] = m_new;
+            }
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[e] = exp2f(x[e] - m_run[nt][e & 1]);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) l_run[nt][i] = l_run[nt][i] * alpha[i] + p[i] + p[i + 2];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[nt][mt][e] *= alpha[e & 1];
+            pb[nt][0] = movmatrix_t(pack_bf16x2(p[0], p[1]));
+            pb[nt][1] = movmatrix_t(pack_bf16x2(p[2], p[3]));
+        }
+        // O^T[dim][head] += V^T . P^T
+        {
+            const int mi = lane >> 3, rr = lane & 7;
+            const int tok = rr + 8 * (mi >> 1);
+            const bool tail = nvalid < DEC_TILE;
+            const int t_lo = 2 * q4, t_hi = 8 + 2 * q4;  // tokens of this lane's A halves
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int chunk = (mt & 3) * 2 + (mi & 1);
+                uint32_t v0, v1, v2, v3;
+                ldsm_x4_t(sV + (mt >> 2) * BOX_BYTES + swz128(tok, chunk), v0, v1, v2, v3);
+                if (tail) {
+                    const uint32_t mlo = (t_lo < nvalid ? 0x0000ffffu : 0u) | (t_lo + 1 < nvalid ? 0xffff0000u : 0u);
+                    const uint32_t mhi = (t_hi < nvalid ? 0x0000ffffu : 0u) | (t_hi + 1 < nvalid ? 0xffff0000u : 0u);
+                    v0 &= mlo;
+                    v1 &= mlo;
+                    v2 &= mhi;
+                    v3 &= mhi;
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc[nt][mt], v0, v1, v2, v3, pb[nt][0], pb[nt][1]);
+            }
+        }
+        __syncwarp();  // every lane is done with this stage before it is refilled
+        ++consumed;
+    }
+
+    if (failed) {
+        // a load did not arrive in time: report, let every issued load land, write no partial
+        if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
+        for (uint32_t i = consumed; i < issued; ++i)
+            (void)mbar_wait_bounded(bar0 + 8u * (i % DEC_STAGES), (i / DEC_STAGES) & 1u);
+        for (int64_t r = row_first; r <= row_last; ++r) write_empty(r);
+        return;
+    }
+    if (cur_row >= 0) {
+        flush(cur_row);
+        flushed_to = cur_row;
+    }
+    for (int64_t r = flushed_to + 1; r <= row_last; ++r) write_empty(r);
+}
+
+// Merge: one warp per (row, query head of the group).
+template <int DV>
+__global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t item = (int64_t)blockIdx.x * 8 + warp;
+    const int64_t rows = (int64_t)a.B * a.Hkv;
+    if (item >= rows * a.G) return;
+    const int64_t r = item / a.G;
+    const int g = static_cast<int>(item % a.G);
+    const int64_t c_lo = chunk_of(r * a.units_per_row, a.units, a.chunks);
+    const int64_t c_hi = chunk_of((r + 1) * a.units_per_row - 1, a.units, a.chunks);
+    float M = -INFINITY;
+    for (int64_t cc = c_lo; cc <= c_hi; ++cc) M = fmaxf(M, a.ml_part[((r + cc) * a.G + g) * 2]);
+    constexpr int PER = DV / 32;  // dims per lane
+    float o[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) o[i] = 0.f;
+    float lsum = 0.f;
+    if (M != -INFINITY) {
+        for (int64_t cc = c_lo; cc <= c_hi; ++cc) {
+            const float *ml = a.ml_part + ((r + cc) * a.G + g) * 2;
+            const float m = ml[0];
+            if (m == -INFINITY) continue;
+            const float w = exp2f(m - M);
+            lsum += w * ml[1];
+            const float *op = a.o_part + ((r + cc) * a.G + g) * DV + lane * PER;
+#pragma unroll
+            for (int i = 0; i < PER; i += 2) {
+                const float2 v = *reinterpret_cast<const float2 *>(op + i);
+                o[i] += w * v.x;
+                o[i + 1] += w * v.y;
+            }
+        }
+    }
+    const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);
+    const size_t head = (size_t)b * a.Hq + (size_t)h * a.G + g;
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    __nv_bfloat16 *dst = a.out + head * DV + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; i += 2)
+        *reinterpret_cast<uint32_t *>(dst + i) = pack_bf16x2(o[i] * inv, o[i + 1] * inv);
+    if (a.lse && lane == 0) a.lse[head] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+template <int D, int NT>
+static cudaError_t launch_gqa_dn(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                                 int grid, cudaStream_t s, bool pdl) {
+    constexpr int STAGE_BYTES = 2 * DEC_TILE * D * 2;
+    const size_t smem = 1024 + (size_t)DEC_WARPS * DEC_STAGES * (STAGE_BYTES + 8 + sizeof(TileMeta));
+    auto kern = k_decode_gqa<D, NT>;
+    static std::atomic<unsigned long long> done;
+    cudaError_t e = ensure_smem_limit(kern, (int)smem, done);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3(grid), dim3(DEC_WARPS * 32), smem, s, pdl, tmK, tmV, a);
+}
+
+cudaError_t launch_decode_gqa(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                              int grid, cudaStream_t s, bool pdl) {
+    const int nt = (a.G + 7) / 8;
+    if (a.Dqk == 128 && nt == 1) return launch_gqa_dn<128, 1>(a, tmK, tmV, grid, s, pdl);
+    if (a.Dqk == 128 && nt == 2) return launch_gqa_dn<128, 2>(a, tmK, tmV, grid, s, pdl);
+    if (a.Dqk == 64 && nt == 1) return launch_gqa_dn<64, 1>(a, tmK, tmV, grid, s, pdl);
+    if (a.Dqk == 64 && nt == 2) return launch_gqa_dn<64, 2>(a, tmK, tmV, grid, s, pdl);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl) {
+    const int64_t items = (int64_t)a.B * a.Hkv * a.G;
+    const dim3 grid((unsigned)((items + 7) / 8));
+    switch (a.Dv) {
+        case 64: return launch_k(k_merge<64>, grid, dim3(256), 0, s, pdl, a);
+        case 128: return launch_k(k_merge<128>, grid, dim3(256), 0, s, pdl, a);
+        case 512: return launch_k(k_merge<512>, grid, dim3(256), 0, s, pdl, a);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace vx

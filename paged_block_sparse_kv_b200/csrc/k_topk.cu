@@ -1,0 +1,289 @@
+// k_topk.cu -- top-k pages per (request, KV head) row of scores.
+//
+// Vortex paper note, section 系统设计 3: radix top-k, the bottleneck of the indexer
+// stage, with stochastic early termination and remapping as the faster approximate
+// form (its kernel-ablation section reports recall@k > 0.97 for that form).
+//
+// One 1024-thread block per row.  Scores become order-preserving uint32 keys (-0.0
+// folded onto +0.0), kept in shared memory when the row fits.
+//   exact:  MSB-first radix select, 8-bit digits, 256-bin shared histograms; the digit
+//           holding the k-th largest key is found with a warp suffix scan; the search
+//           stops early once the boundary bucket holds exactly the slots left.
+//   approx: fp32 remap of each score to a 12-bit code between the row's min and max,
+//           one 4096-bin histogram, the boundary code b* from a block suffix scan, no
+//           refinement: the slots left are filled from code b* in cyclic page order from
+//           a SplitMix64-drawn offset.
+// Both finish with an ordered compaction (two block-wide exclusive scans over
+// contiguous per-thread runs), so the chosen pages come out in ascending page order and
+// boundary ties go to the lower page index (exact) or to the first pages after the
+// drawn offset (approx).
+#include "vx_internal.h"
+
+namespace vx {
+
+__device__ __forceinline__ uint32_t order_key(float s) {
+    uint32_t f = __float_as_uint(s);
+    if (f == 0x80000000u) f = 0u;  // -0.0 ties with +0.0
+    return (f & 0x80000000u) ? ~f : (f | 0x80000000u);
+}
+
+// SplitMix64 (Steele, Lea and Flood 2014): draw number i of the generator seeded with seed.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t i) {
+    uint64_t z = seed + (i + 1ull) * 0x9e3779b97f4a7c15ull;
+    z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ull;
+    z = (z ^ (z >> 27)) * 0x94d049bb133111ebull;
+    return z ^ (z >> 31);
+}
+
+// Block-wide exclusive scan of one int per thread (TOPK_THREADS threads); also returns
+// the total.  `tmp` holds 32 ints of shared memory.  Contains __syncthreads.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *tmp, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(FULL, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) tmp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = tmp[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(FULL, w, off);
+            if (lane >= off) w += y;
+        }
+        tmp[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    total = tmp[31];
+    const int before = (warp > 0 ? tmp[warp - 1] : 0) + x - v;
+    __syncthreads();  // tmp may be reused right after
+    return before;
+}
+
+struct TopkShared {
+    int hist[1 << APPROX_BITS];
+    int scan_tmp[32];
+    int bcast[4];
+    float fmin[32], fmax[32];
+};
+
+template <bool APPROX>
+__global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
+    pdl_launch_dependents();
+    pdl_wait();  // the scores are written by the previous kernel
+    __shared__ TopkShared sh;
+    extern __shared__ uint32_t skeys[];  // a.smem_keys entries
+    const int b = blockIdx.y, h = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int32_t *out = a.sel + ((size_t)b * a.Hkv + h) * a.k;
+    const float *row = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages;
+    const int32_t L = a.seq_lens[b];
+    if (L < 1 || L > a.max_pages * a.P) {
+        for (int i = tid; i < a.k; i += TOPK_THREADS) out[i] = -1;
+        if (tid == 0 && h == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
+        return;
+    }
+    const int n = ceil_div(L, a.P);
+    const int keff = min(a.k, n);
+    if (keff == n) {  // every page is chosen
+        for (int i = tid; i < a.k; i += TOPK_THREADS) out[i] = i < n ? i : -1;
+        return;
+    }
+    const bool in_smem = n <= a.smem_keys;
+
+    // per-thread contiguous run [r0, r1) used by the ordered compaction
+    const int per = ceil_div(n, TOPK_THREADS);
+    const int r0 = min(n, tid * per), r1 = min(n, r0 + per);
+
+    // -------- key of page j: radix key (exact) or remap code (approx)
+    uint32_t prefix = 0, mask = 0;  // exact: chosen iff (key & mask) > prefix, or == and rank < remaining
+    int remaining = keff;           // slots to take from the boundary bucket
+    int offset = 0;                 // approx: start of the cyclic fill
+    float lo = 0.f, scale = 0.f;
+    bool flat = false;
+
+    if constexpr (!APPROX) {
+        if (in_smem)
+            for (int j = tid; j < n; j += TOPK_THREADS) skeys[j] = order_key(row[j]);
+        __syncthreads();
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int i = tid; i < 256; i += TOPK_THREADS) sh.hist[i] = 0;
+            __syncthreads();
+            for (int j = tid; j < n; j += TOPK_THREADS) {
+                const uint32_t key = in_smem ? skeys[j] : order_key(row[j]);
+                if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // lane owns digits [8*lane, 8*lane+8); suffix sums from the top digit down
+                int c[8], own = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    c[i] = sh.hist[lane * 8 + i];
+                    own += c[i];
+                }
+                int suf = own;  // inclusive suffix over lanes >= lane
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_down_sync(FULL, suf, off);
+                    if (lane + off < 32) suf += y;
+                }
+                int above = suf - own;  // digits owned by higher lanes
+#pragma unroll
+                for (int i = 7; i >= 0; --i) {
+                    if (above < remaining && above + c[i] >= remaining) {
+                        sh.bcast[0] = lane * 8 + i;
+                        sh.bcast[1] = above;
+                        sh.bcast[2] = c[i];
+                    }
+                    above += c[i];
+                }
+            }
+            __syncthreads();
+            const int digit = sh.bcast[0], above = sh.bcast[1], cnt = sh.bcast[2];
+            remaining -= above;
+            prefix |= static_cast<uint32_t>(digit) << shift;
+            mask |= 0xffu << shift;
+            __syncthreads();
+            if (cnt == remaining) break;  // the whole boundary bucket is taken
+        }
+    } else {
+        // row min / max
+        float mn = INFINITY, mx = -INFINITY;
+        for (int j = tid; j < n; j += TOPK_THREADS) {
+            const float s = row[j];
+            mn = fminf(mn, s);
+            mx = fmaxf(mx, s);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(FULL, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, off));
+        }
+        if (lane == 0) {
+            sh.fmin[warp] = mn;
+            sh.fmax[warp] = mx;
+        }
+        for (int i = tid; i < (1 << APPROX_BITS); i += TOPK_THREADS) sh.hist[i] = 0;
+        __syncthreads();
+        mn = sh.fmin[0];
+        mx = sh.fmax[0];
+        for (int w = 1; w < TOPK_THREADS / 32; ++w) {
+            mn = fminf(mn, sh.fmin[w]);
+            mx = fmaxf(mx, sh.fmax[w]);
+        }
+        lo = mn;
+        const float range = __fsub_rn(mx, mn);
+        scale = __fdiv_rn(static_cast<float>(1 << APPROX_BITS), range);
+        flat = !(mx > mn) || isinf(scale);
+        for (int j = tid; j < n; j += TOPK_THREADS) {
+            uint32_t code = 0;
+            if (!flat) {
+                const float t = __fmul_rn(__fsub_rn(row[j], lo), scale);
+                const float f = floorf(t);
+                code = f >= float((1 << APPROX_BITS) - 1) ? (1u << APPROX_BITS) - 1 : static_cast<uint32_t>(f);
+            }
+            if (in_smem) skeys[j] = code;
+            atomicAdd(&sh.hist[code], 1);
+        }
+        __syncthreads();
+        // boundary code: suffix scan of 4096 bins, 4 per thread, highest bins first
+        constexpr int BPT = (1 << APPROX_BITS) / TOPK_THREADS;
+        const int base = (TOPK_THREADS - 1 - tid) * BPT;  // thread 0 owns the top bins
+        int own = 0;
+#pragma unroll
+        for (int i = 0; i < BPT; ++i) own += sh.hist[base + i];
+        int total;
+        int above = block_exclusive_scan(own, sh.scan_tmp, total);
+#pragma unroll
+        for (int i = BPT - 1; i >= 0; --i) {
+            const int c = sh.hist[base + i];
+            if (above < keff && above + c >= keff) {
+                sh.bcast[0] = base + i;
+                sh.bcast[1] = above;
+            }
+            above += c;
+        }
+        __syncthreads();
+        prefix = static_cast<uint32_t>(sh.bcast[0]);
+        mask = 0xffffffffu;
+        remaining = keff - sh.bcast[1];
+        offset = static_cast<int>(splitmix64(a.seed, (uint64_t)b * a.Hkv + h) % (uint64_t)n);
+    }
+
+    auto key_of = [&](int j) -> uint32_t {
+        if (in_smem) return skeys[j];
+        if constexpr (APPROX) {
+            if (flat) return 0u;
+            const float f = floorf(__fmul_rn(__fsub_rn(row[j], lo), scale));
+            return f >= float((1 << APPROX_BITS) - 1) ? (1u << APPROX_BITS) - 1 : static_cast<uint32_t>(f);
+        } else {
+            return order_key(row[j]);
+        }
+    };
+
+    // -------- ordered compaction
+    // pass 1: rank of each boundary-bucket member among the members in page order
+    int eq_local = 0, eq_before_offset_local = 0;
+    for (int j = r0; j < r1; ++j) {
+        if ((key_of(j) & mask) == prefix) {
+            ++eq_local;
+            if (j < offset) ++eq_before_offset_local;
+        }
+    }
+    int eq_total;
+    const int eq_before = block_exclusive_scan(eq_local, sh.scan_tmp, eq_total);
+    int eq_before_offset = 0;
+    if constexpr (APPROX) {
+        int tmp_total;
+        block_exclusive_scan(eq_before_offset_local, sh.scan_tmp, tmp_total);
+        eq_before_offset = tmp_total;  // members with page index < offset
+    }
+    // pass 2: chosen flags, counted per run
+    auto chosen = [&](uint32_t key, int j, int eq_rank) -> bool {
+        const uint32_t mk = key & mask;
+        if (mk > prefix) return true;
+        if (mk != prefix) return false;
+        int r = eq_rank;
+        if constexpr (APPROX) r = (j >= offset) ? eq_rank - eq_before_offset : eq_total - eq_before_offset + eq_rank;
+        return r < remaining;
+    };
+    int sel_local = 0;
+    {
+        int eq_rank = eq_before;
+        for (int j = r0; j < r1; ++j) {
+            const uint32_t key = key_of(j);
+            if (chosen(key, j, eq_rank)) ++sel_local;
+            if ((key & mask) == prefix) ++eq_rank;
+        }
+    }
+    int sel_total;
+    int pos = block_exclusive_scan(sel_local, sh.scan_tmp, sel_total);
+    {
+        int eq_rank = eq_before;
+        for (int j = r0; j < r1; ++j) {
+            const uint32_t key = key_of(j);
+            if (chosen(key, j, eq_rank)) {
+                if (pos < a.k) out[pos] = j;
+                ++pos;
+            }
+            if ((key & mask) == prefix) ++eq_rank;
+        }
+    }
+    for (int i = sel_total + tid; i < a.k; i += TOPK_THREADS) out[i] = -1;
+}
+
+cudaError_t launch_topk(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
+    dim3 grid(a.Hkv, a.B);
+    const size_t smem = sizeof(uint32_t) * (size_t)a.smem_keys;
+    auto kern = mode == 0 ? k_topk<false> : k_topk<true>;
+    static std::atomic<unsigned long long> done[2];
+    cudaError_t e = ensure_smem_limit(kern, (int)(sizeof(uint32_t) * TOPK_SMEM_KEYS), done[mode]);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, grid, dim3(TOPK_THREADS), smem, s, pdl, a);
+}
+
+}  // namespace vx

@@ -1,0 +1,471 @@
+// vx_api.cu -- the C ABI of libvx (include/vx.h): validation, planning, launches.
+//
+// Host validation runs before anything is launched and touches no CUDA state, so bad
+// arguments fail the same way with or without a GPU.  Workload planning (paper note,
+// section 系统设计 3) picks the split count from the SM count: one persistent block of
+// DEC_WARPS worker warps per SM for GQA, two blocks per SM for MLA.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "vx_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+vx_status fail(vx_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+vx_status fail(vx_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+vx_status cuda_fail(cudaError_t e, const char *where) {
+    return fail(VX_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// ------------------------------------------------------------------ validation
+
+vx_status check_geometry(const vx_geometry *g) {
+    if (!g) return fail(VX_ERR_INVALID_ARG, "geometry is NULL");
+    if (g->batch < 1) return fail(VX_ERR_INVALID_ARG, "batch %d < 1", g->batch);
+    if (g->num_kv_heads < 1 || g->num_q_heads < 1)
+        return fail(VX_ERR_INVALID_ARG, "head counts must be >= 1 (q %d, kv %d)", g->num_q_heads, g->num_kv_heads);
+    if (g->num_q_heads % g->num_kv_heads)
+        return fail(VX_ERR_INVALID_ARG, "num_q_heads %d is not a multiple of num_kv_heads %d", g->num_q_heads,
+                    g->num_kv_heads);
+    if (g->num_pool_pages < 1) return fail(VX_ERR_INVALID_ARG, "num_pool_pages must be >= 1");
+    if (g->page_size < 1 || g->head_dim_qk < 1 || g->head_dim_v < 1)
+        return fail(VX_ERR_INVALID_ARG, "page_size and head dims must be >= 1");
+    if (g->num_pool_pages * (int64_t)g->num_kv_heads > INT32_MAX)
+        return fail(VX_ERR_INVALID_ARG, "num_pool_pages * num_kv_heads overflows int32");
+    const int G = g->num_q_heads / g->num_kv_heads;
+    if (g->page_size != 16 && g->page_size != 32 && g->page_size != 64)
+        return fail(VX_ERR_UNSUPPORTED, "page_size %d not built (16, 32, 64)", g->page_size);
+    if (g->mla_shared_kv) {
+        if (g->num_kv_heads != 1 || g->head_dim_qk != 576 || g->head_dim_v != 512)
+            return fail(VX_ERR_UNSUPPORTED, "MLA geometry must be 1 KV head, head_dim_qk 576, head_dim_v 512");
+        if (G > 16) return fail(VX_ERR_UNSUPPORTED, "MLA supports at most 16 query heads (got %d)", G);
+    } else {
+        if (g->head_dim_qk != g->head_dim_v) return fail(VX_ERR_UNSUPPORTED, "GQA needs head_dim_qk == head_dim_v");
+        if (g->head_dim_qk != 64 && g->head_dim_qk != 128)
+            return fail(VX_ERR_UNSUPPORTED, "GQA head_dim %d not built (64, 128)", g->head_dim_qk);
+        if (G > 16) return fail(VX_ERR_UNSUPPORTED, "GQA group size %d > 16 not built", G);
+        if (g->num_kv_heads * g->head_dim_qk > 1024)
+            return fail(VX_ERR_UNSUPPORTED, "num_kv_heads * head_dim %d > 1024 not built",
+                        g->num_kv_heads * g->head_dim_qk);
+    }
+    return VX_OK;
+}
+
+vx_status check_max_pages(const vx_geometry *g, int32_t max_pages) {
+    if (max_pages < 1) return fail(VX_ERR_INVALID_ARG, "max_pages must be >= 1");
+    if ((int64_t)max_pages * g->page_size > INT32_MAX)
+        return fail(VX_ERR_INVALID_ARG, "max_pages * page_size overflows int32");
+    return VX_OK;
+}
+
+vx_status check_geo(const vx_geometry *g, const vx_page_table *t) {
+    vx_status s = check_geometry(g);
+    if (s != VX_OK) return s;
+    if (!t) return fail(VX_ERR_INVALID_ARG, "page table is NULL");
+    if (!t->page_ptr || !t->page_indices || !t->seq_lens)
+        return fail(VX_ERR_INVALID_ARG, "page table arrays must not be NULL");
+    if (!al4(t->page_ptr) || !al4(t->page_indices) || !al4(t->seq_lens))
+        return fail(VX_ERR_INVALID_ARG, "page table arrays must be 4-byte aligned");
+    return check_max_pages(g, t->max_pages);
+}
+
+vx_status check_ptr(const void *p, const char *name, bool can_be_null = false) {
+    if (!p) return can_be_null ? VX_OK : fail(VX_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!al16(p)) return fail(VX_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return VX_OK;
+}
+
+#define VX_TRY(x)                          \
+    do {                                   \
+        vx_status _s = (x);                \
+        if (_s != VX_OK) return _s;        \
+    } while (0)
+
+// ------------------------------------------------------------------ device facts
+
+int sm_count_current(int *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    static int cache[64] = {0};
+    if (dev < 64 && cache[dev]) {
+        *out = cache[dev];
+        return 0;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return -1;
+    if (dev < 64) cache[dev] = n;
+    *out = n;
+    return 0;
+}
+
+// ------------------------------------------------------------------ planning
+
+struct Plan {
+    int64_t rows, units, units_per_row;
+    int32_t tiles_per_page, chunks, grid;
+    int G;
+    bool mla;
+};
+
+constexpr int MLA_BLOCKS_PER_SM = 2;
+
+vx_status plan(const vx_geometry *g, int32_t k, int32_t num_splits, Plan *p) {
+    p->mla = g->mla_shared_kv != 0;
+    p->G = g->num_q_heads / g->num_kv_heads;
+    p->rows = (int64_t)g->batch * g->num_kv_heads;
+    p->tiles_per_page = g->page_size / vx::DEC_TILE;
+    p->units_per_row = (int64_t)k * p->tiles_per_page;
+    p->units = p->rows * p->units_per_row;
+    int64_t w = num_splits;
+    if (w <= 0) {
+        int sms = 0;
+        if (sm_count_current(&sms) != 0) return fail(VX_ERR_CUDA, "cannot query the current device's SM count");
+        w = p->mla ? (int64_t)sms * MLA_BLOCKS_PER_SM : (int64_t)sms * vx::DEC_WARPS;
+    }
+    if (w > p->units) w = p->units;
+    if (w < 1) w = 1;
+    if (w > INT32_MAX / 2) return fail(VX_ERR_INVALID_ARG, "num_splits too large");
+    p->chunks = static_cast<int32_t>(w);
+    p->grid = p->mla ? p->chunks : (p->chunks + vx::DEC_WARPS - 1) / vx::DEC_WARPS;
+    return VX_OK;
+}
+
+// workspace layout, every region 256-byte aligned
+struct WsLayout {
+    size_t scores, sel, o_part, ml_part, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(const vx_geometry *g, int32_t max_pages, int32_t k, const Plan &p) {
+    WsLayout l;
+    const size_t slots = (size_t)(p.rows + p.chunks);
+    l.o_part = 0;
+    l.ml_part = l.o_part + up256(slots * p.G * g->head_dim_v * sizeof(float));
+    l.scores = l.ml_part + up256(slots * p.G * 2 * sizeof(float));
+    l.sel = l.scores + up256((size_t)p.rows * max_pages * sizeof(float));
+    l.total = l.sel + up256((size_t)p.rows * k * sizeof(int32_t));
+    return l;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// 3-D view [pages * heads][page_size][dim] of a bf16 cache, boxes of 64 dims x box_rows
+// tokens x 1 page-head, 128-byte swizzle.
+vx_status make_cache_map(CUtensorMap *map, const void *ptr, int dim, int page_size, int64_t page_heads,
+                         int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)page_size, (cuuint64_t)page_heads};
+    cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * 2 * page_size};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return VX_OK;
+}
+
+// ------------------------------------------------------------------ shared launch pieces
+
+vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q, const void *k_cache,
+                    const void *v_cache, const int32_t *sel, int32_t k, float sm_scale, const Plan &p,
+                    const WsLayout &l, void *ws, void *out, float *lse, int32_t *err, cudaStream_t s, bool pdl) {
+    vx::DecodeArgs a{};
+    a.page_ptr = t->page_ptr;
+    a.page_indices = t->page_indices;
+    a.seq_lens = t->seq_lens;
+    a.sel = sel;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.o_part = reinterpret_cast<float *>(static_cast<char *>(ws) + l.o_part);
+    a.ml_part = reinterpret_cast<float *>(static_cast<char *>(ws) + l.ml_part);
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.err = err;
+    a.B = g->batch;
+    a.Hq = g->num_q_heads;
+    a.Hkv = g->num_kv_heads;
+    a.G = p.G;
+    a.Dqk = g->head_dim_qk;
+    a.Dv = g->head_dim_v;
+    a.P = g->page_size;
+    a.max_pages = t->max_pages;
+    a.k = k;
+    a.tiles_per_page = p.tiles_per_page;
+    a.num_pool_pages = g->num_pool_pages;
+    a.units = p.units;
+    a.units_per_row = p.units_per_row;
+    a.chunks = p.chunks;
+    const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)g->head_dim_qk);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    const int64_t page_heads = g->num_pool_pages * g->num_kv_heads;
+    cudaError_t e;
+    if (p.mla) {
+        CUtensorMap tmK;
+        VX_TRY(make_cache_map(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::DEC_TILE));
+        e = vx::launch_decode_mla(a, tmK, p.grid, s, pdl);
+    } else {
+        CUtensorMap tmK, tmV;
+        VX_TRY(make_cache_map(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::DEC_TILE));
+        VX_TRY(make_cache_map(&tmV, v_cache, g->head_dim_v, g->page_size, page_heads, vx::DEC_TILE));
+        e = vx::launch_decode_gqa(a, tmK, tmV, p.grid, s, pdl);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
+    e = vx::launch_merge(a, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+    return VX_OK;
+}
+
+vx::ScoreArgs score_args(const vx_geometry *g, const vx_page_table *t, const void *q, const void *centroids,
+                         int32_t score_dims, float *scores, int32_t *err) {
+    vx::ScoreArgs a{};
+    a.page_ptr = t->page_ptr;
+    a.page_indices = t->page_indices;
+    a.seq_lens = t->seq_lens;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.centroids = static_cast<const __nv_bfloat16 *>(centroids);
+    a.scores = scores;
+    a.err = err;
+    a.B = g->batch;
+    a.Hq = g->num_q_heads;
+    a.Hkv = g->num_kv_heads;
+    a.G = g->num_q_heads / g->num_kv_heads;
+    a.Dqk = g->head_dim_qk;
+    a.P = g->page_size;
+    a.max_pages = t->max_pages;
+    a.score_dims = score_dims > 0 ? score_dims : g->head_dim_qk;
+    a.num_pool_pages = g->num_pool_pages;
+    return a;
+}
+
+vx::TopkArgs topk_args(const vx_geometry *g, const vx_page_table *t, const float *scores, int32_t k, uint64_t seed,
+                       int32_t *sel, int32_t *err) {
+    vx::TopkArgs a{};
+    a.seq_lens = t->seq_lens;
+    a.scores = scores;
+    a.sel = sel;
+    a.err = err;
+    a.B = g->batch;
+    a.Hkv = g->num_kv_heads;
+    a.P = g->page_size;
+    a.max_pages = t->max_pages;
+    a.k = k;
+    a.smem_keys = t->max_pages < vx::TOPK_SMEM_KEYS ? t->max_pages : vx::TOPK_SMEM_KEYS;
+    a.seed = seed;
+    return a;
+}
+
+vx_status check_score_dims(const vx_geometry *g, int32_t score_dims) {
+    if (score_dims < 0 || score_dims > g->head_dim_qk || (score_dims % 8) != 0)
+        return fail(VX_ERR_INVALID_ARG, "score_dims %d must be 0 or a multiple of 8 in [8, head_dim_qk]", score_dims);
+    return VX_OK;
+}
+
+vx_status check_k_mode(int32_t k, int32_t mode) {
+    if (k < 1) return fail(VX_ERR_INVALID_ARG, "k %d < 1", k);
+    if (mode != 0 && mode != 1) return fail(VX_ERR_INVALID_ARG, "mode %d must be 0 (exact) or 1 (approximate)", mode);
+    return VX_OK;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+const char *vx_status_string(vx_status s) {
+    switch (s) {
+        case VX_OK: return "VX_OK";
+        case VX_ERR_INVALID_ARG: return "VX_ERR_INVALID_ARG";
+        case VX_ERR_UNSUPPORTED: return "VX_ERR_UNSUPPORTED";
+        case VX_ERR_WORKSPACE: return "VX_ERR_WORKSPACE";
+        case VX_ERR_CUDA: return "VX_ERR_CUDA";
+    }
+    return "VX_UNKNOWN_STATUS";
+}
+
+const char *vx_last_error(void) { return g_last_error.c_str(); }
+
+const char *vx_version(void) { return "libvx 0.1 (sm_100a)"; }
+
+size_t vx_workspace_size(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits) {
+    if (check_geometry(geo) != VX_OK || check_max_pages(geo, max_pages) != VX_OK) return 0;
+    if (k < 1) {
+        fail(VX_ERR_INVALID_ARG, "k %d < 1", k);
+        return 0;
+    }
+    Plan p;
+    if (plan(geo, k, num_splits, &p) != VX_OK) return 0;
+    return ws_layout(geo, max_pages, k, p).total;
+}
+
+int32_t vx_planned_splits(const vx_geometry *geo, int32_t max_pages, int32_t k) {
+    if (check_geometry(geo) != VX_OK || check_max_pages(geo, max_pages) != VX_OK) return 0;
+    if (k < 1) {
+        fail(VX_ERR_INVALID_ARG, "k %d < 1", k);
+        return 0;
+    }
+    Plan p;
+    if (plan(geo, k, 0, &p) != VX_OK) return 0;
+    return p.chunks;
+}
+
+vx_status vx_centroid_update(const vx_geometry *geo, const vx_page_table *table, void *k_cache, void *v_cache,
+                             void *centroids, const void *k_new, const void *v_new, const int32_t *first_pos,
+                             int32_t *err, void *stream) {
+    VX_TRY(check_geo(geo, table));
+    VX_TRY(check_ptr(k_cache, "k_cache"));
+    VX_TRY(check_ptr(centroids, "centroids"));
+    const bool append = k_new != nullptr;
+    if (append) {
+        VX_TRY(check_ptr(k_new, "k_new"));
+        if (!geo->mla_shared_kv) {
+            VX_TRY(check_ptr(v_cache, "v_cache"));
+            VX_TRY(check_ptr(v_new, "v_new"));
+        }
+    }
+    if (first_pos && !al4(first_pos)) return fail(VX_ERR_INVALID_ARG, "first_pos must be 4-byte aligned");
+    if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
+    vx::CentroidArgs a{};
+    a.page_ptr = table->page_ptr;
+    a.page_indices = table->page_indices;
+    a.seq_lens = table->seq_lens;
+    a.first_pos = append ? nullptr : first_pos;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.centroids = centroids;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.err = err;
+    a.B = geo->batch;
+    a.Hkv = geo->num_kv_heads;
+    a.Dqk = geo->head_dim_qk;
+    a.Dv = geo->head_dim_v;
+    a.P = geo->page_size;
+    a.max_pages = table->max_pages;
+    a.mla_shared_kv = geo->mla_shared_kv;
+    a.num_pool_pages = geo->num_pool_pages;
+    cudaError_t e = vx::launch_centroid(a, append, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "centroid launch");
+    return VX_OK;
+}
+
+vx_status vx_score_pages(const vx_geometry *geo, const vx_page_table *table, const void *q, const void *centroids,
+                         int32_t score_dims, float *scores, int32_t *err, void *stream) {
+    VX_TRY(check_geo(geo, table));
+    VX_TRY(check_ptr(q, "q"));
+    VX_TRY(check_ptr(centroids, "centroids"));
+    VX_TRY(check_ptr(scores, "scores"));
+    VX_TRY(check_score_dims(geo, score_dims));
+    if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
+    cudaError_t e = vx::launch_score(score_args(geo, table, q, centroids, score_dims, scores, err),
+                                     static_cast<cudaStream_t>(stream), false);
+    if (e != cudaSuccess) return cuda_fail(e, "score launch");
+    return VX_OK;
+}
+
+vx_status vx_topk_pages(const vx_geometry *geo, const vx_page_table *table, const float *scores, int32_t k,
+                        int32_t mode, uint64_t seed, int32_t *sel, int32_t *err, void *stream) {
+    VX_TRY(check_geo(geo, table));
+    VX_TRY(check_ptr(scores, "scores"));
+    VX_TRY(check_ptr(sel, "sel"));
+    VX_TRY(check_k_mode(k, mode));
+    if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
+    cudaError_t e = vx::launch_topk(topk_args(geo, table, scores, k, seed, sel, err), mode,
+                                    static_cast<cudaStream_t>(stream), false);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+    return VX_OK;
+}
+
+vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, const void *q, const void *k_cache,
+                           const void *v_cache, const int32_t *sel, int32_t k, float sm_scale, int32_t num_splits,
+                           void *out, float *lse, void *ws, size_t ws_bytes, int32_t *err, void *stream) {
+    VX_TRY(check_geo(geo, table));
+    VX_TRY(check_ptr(q, "q"));
+    VX_TRY(check_ptr(k_cache, "k_cache"));
+    if (!geo->mla_shared_kv) VX_TRY(check_ptr(v_cache, "v_cache"));
+    VX_TRY(check_ptr(sel, "sel"));
+    VX_TRY(check_ptr(out, "out"));
+    VX_TRY(check_ptr(lse, "lse", true));
+    VX_TRY(check_k_mode(k, 0));
+    if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
+    if (!std::isfinite(sm_scale)) return fail(VX_ERR_INVALID_ARG, "sm_scale must be finite");
+    Plan p;
+    VX_TRY(plan(geo, k, num_splits, &p));
+    const WsLayout l = ws_layout(geo, table->max_pages, k, p);
+    if (!ws || !al16(ws)) return fail(VX_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+    if (ws_bytes < l.total)
+        return fail(VX_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, l.total);
+    return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, ws, out, lse, err,
+                     static_cast<cudaStream_t>(stream), false);
+}
+
+vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *table, const void *q, const void *k_cache,
+                               const void *v_cache, const void *centroids, int32_t k, int32_t mode, uint64_t seed,
+                               float sm_scale, int32_t score_dims, int32_t num_splits, void *out, float *lse,
+                               float *scores_out, int32_t *sel_out, void *ws, size_t ws_bytes, int32_t *err,
+                               void *stream) {
+    VX_TRY(check_geo(geo, table));
+    VX_TRY(check_ptr(q, "q"));
+    VX_TRY(check_ptr(k_cache, "k_cache"));
+    if (!geo->mla_shared_kv) VX_TRY(check_ptr(v_cache, "v_cache"));
+    VX_TRY(check_ptr(centroids, "centroids"));
+    VX_TRY(check_ptr(out, "out"));
+    VX_TRY(check_ptr(lse, "lse", true));
+    VX_TRY(check_ptr(scores_out, "scores_out", true));
+    VX_TRY(check_ptr(sel_out, "sel_out", true));
+    VX_TRY(check_k_mode(k, mode));
+    VX_TRY(check_score_dims(geo, score_dims));
+    if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
+    if (!std::isfinite(sm_scale)) return fail(VX_ERR_INVALID_ARG, "sm_scale must be finite");
+    Plan p;
+    VX_TRY(plan(geo, k, num_splits, &p));
+    const WsLayout l = ws_layout(geo, table->max_pages, k, p);
+    if (!ws || !al16(ws)) return fail(VX_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+    if (ws_bytes < l.total)
+        return fail(VX_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, l.total);
+    float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<char *>(ws) + l.scores);
+    int32_t *sel = sel_out ? sel_out : reinterpret_cast<int32_t *>(static_cast<char *>(ws) + l.sel);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = vx::launch_score(score_args(geo, table, q, centroids, score_dims, scores, err), s, false);
+    if (e != cudaSuccess) return cuda_fail(e, "score launch");
+    e = vx::launch_topk(topk_args(geo, table, scores, k, seed, sel, err), mode, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+    return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, ws, out, lse, err, s, true);
+}
+
+}  // extern "C"

@@ -1,0 +1,130 @@
+// vx_internal.h -- argument blocks and launch entry points shared by the libvx sources.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <utility>
+
+#include "vx_common.cuh"
+
+namespace vx {
+
+// ------------------------------------------------------------------ tunables
+constexpr int CEN_WARPS = 8;             // centroid rebuild: warps per block
+constexpr int CEN_PAGES_PER_BLOCK = 16;  // centroid rebuild: pages per block
+constexpr int SCORE_WARPS = 8;           // scoring: warps per block
+constexpr int SCORE_UNROLL = 4;          // scoring: pages in flight per warp
+constexpr int SCORE_PAGES_PER_BLOCK = SCORE_WARPS * SCORE_UNROLL * 2;
+constexpr int TOPK_THREADS = 1024;       // top-k: one block per (request, KV head) row
+constexpr int TOPK_SMEM_KEYS = 12288;    // rows up to this many pages keep their keys in smem
+constexpr int APPROX_BITS = 12;          // approximate top-k remap width
+constexpr int DEC_WARPS = 8;             // GQA decode: worker warps per block
+constexpr int DEC_STAGES = 3;            // GQA decode: 16-token tiles in flight per warp
+constexpr int DEC_TILE = 16;             // tokens per tile (one mma M or K step)
+
+// ------------------------------------------------------------------ argument blocks
+struct TableArgs {
+    const int32_t *page_ptr;
+    const int32_t *page_indices;
+    const int32_t *seq_lens;
+};
+
+struct CentroidArgs {
+    const int32_t *page_ptr, *page_indices, *seq_lens, *first_pos;
+    void *k_cache, *v_cache, *centroids;
+    const void *k_new, *v_new;
+    int32_t *err;
+    int32_t B, Hkv, Dqk, Dv, P, max_pages, mla_shared_kv;
+    int64_t num_pool_pages;
+};
+
+struct ScoreArgs {
+    const int32_t *page_ptr, *page_indices, *seq_lens;
+    const __nv_bfloat16 *q, *centroids;
+    float *scores;
+    int32_t *err;
+    int32_t B, Hq, Hkv, G, Dqk, P, max_pages, score_dims;
+    int64_t num_pool_pages;
+};
+
+struct TopkArgs {
+    const int32_t *seq_lens;
+    const float *scores;
+    int32_t *sel;
+    int32_t *err;
+    int32_t B, Hkv, P, max_pages, k, smem_keys;
+    uint64_t seed;
+};
+
+struct DecodeArgs {
+    const int32_t *page_ptr, *page_indices, *seq_lens, *sel;
+    const __nv_bfloat16 *q;
+    float *o_part;   // [slots][G][Dv] unnormalised partial outputs
+    float *ml_part;  // [slots][G][2]  (running max in log2 units, running sum)
+    __nv_bfloat16 *out;
+    float *lse;
+    int32_t *err;
+    int32_t B, Hq, Hkv, G, Dqk, Dv, P, max_pages, k;
+    int32_t tiles_per_page;   // P / DEC_TILE (GQA) or 1 (MLA: one page per unit)
+    int64_t num_pool_pages;
+    int64_t units;            // rows * k * tiles_per_page
+    int64_t units_per_row;    // k * tiles_per_page
+    int32_t chunks;           // split count W
+    float scale_log2;         // sm_scale * log2(e)
+};
+
+// ------------------------------------------------------------------ launches
+cudaError_t launch_centroid(const CentroidArgs &a, bool append, cudaStream_t s);
+cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s, bool pdl);
+cudaError_t launch_topk(const TopkArgs &a, int mode, cudaStream_t s, bool pdl);
+cudaError_t launch_decode_gqa(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                              int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_decode_mla(const DecodeArgs &a, const CUtensorMap &tmK, int grid, cudaStream_t s,
+                              bool pdl);
+cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl);
+
+// Launch with programmatic dependent launch enabled when `pdl` (the kernel must call
+// pdl_wait() before reading what the previous kernel on the stream wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     bool pdl, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute is per
+// device; the first launch on each device sets it).
+template <typename F>
+cudaError_t ensure_smem_limit(F kern, int bytes, std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
+// chunk c of W covers units [c*T/W, (c+1)*T/W)
+__host__ __device__ __forceinline__ int64_t chunk_start(int64_t c, int64_t T, int64_t W) {
+    return (c * T) / W;
+}
+// the chunk holding unit u
+__host__ __device__ __forceinline__ int64_t chunk_of(int64_t u, int64_t T, int64_t W) {
+    return ((u + 1) * W - 1) / T;
+}
+
+}  // namespace vx

@@ -1,0 +1,125 @@
+"""Host side of the C ABI (no GPU needed): the library loads, exports every symbol that
+include/vx.h declares, and rejects bad arguments with the documented status before
+launching anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from paged_block_sparse_kv_b200 import vx
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vx.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vx_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(vx.LIB_PATH):
+        pytest.skip("libvx.so not built")
+    return vx.lib()
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(vx.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", vx.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_no_oracle_in_the_product(L):
+    # the product library links nothing from the oracle
+    out = subprocess.run(["nm", "-D", vx.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    assert "orc_" not in out
+
+
+def _geo(**kw):
+    g = dict(batch=2, num_q_heads=16, num_kv_heads=8, head_dim_qk=128, head_dim_v=128, page_size=16,
+             mla_shared_kv=0, num_pool_pages=100)
+    g.update(kw)
+    return vx.vx_geometry(**g)
+
+
+def _table(max_pages=10, ptr=256):
+    return vx.vx_page_table(ptr, ptr, ptr, max_pages)
+
+
+FAKE = 4096  # an aligned non-NULL address; validation fails before anything dereferences it
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), vx.VX_ERR_INVALID_ARG),
+    (dict(num_q_heads=12, num_kv_heads=8), vx.VX_ERR_INVALID_ARG),
+    (dict(num_pool_pages=0), vx.VX_ERR_INVALID_ARG),
+    (dict(page_size=8), vx.VX_ERR_UNSUPPORTED),
+    (dict(head_dim_qk=96, head_dim_v=96), vx.VX_ERR_UNSUPPORTED),
+    (dict(head_dim_v=64), vx.VX_ERR_UNSUPPORTED),
+    (dict(num_q_heads=8 * 32), vx.VX_ERR_UNSUPPORTED),
+    (dict(mla_shared_kv=1), vx.VX_ERR_UNSUPPORTED),
+    (dict(mla_shared_kv=1, num_kv_heads=1, num_q_heads=32, head_dim_qk=576, head_dim_v=512, page_size=64),
+     vx.VX_ERR_UNSUPPORTED),
+])
+def test_bad_geometry_is_rejected_before_launch(L, kw, status):
+    g = _geo(**kw)
+    t = _table()
+    st = L.vx_score_pages(ctypes.byref(g), ctypes.byref(t), FAKE, FAKE, 0, FAKE, None, None)
+    assert st == status, L.vx_last_error()
+    assert L.vx_last_error().decode()
+    assert L.vx_workspace_size(ctypes.byref(g), 10, 4, 8) == 0
+
+
+def test_bad_pointers_and_sizes(L):
+    g, t = _geo(), _table()
+    gp, tp = ctypes.byref(g), ctypes.byref(t)
+    assert L.vx_score_pages(None, tp, FAKE, FAKE, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_score_pages(gp, None, FAKE, FAKE, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_score_pages(gp, tp, None, FAKE, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_score_pages(gp, tp, FAKE + 2, FAKE, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # misaligned
+    assert L.vx_score_pages(gp, tp, FAKE, FAKE, 12, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # not /8
+    assert L.vx_score_pages(gp, tp, FAKE, FAKE, 136, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # > dqk
+    bad_table = _table(max_pages=0)
+    assert L.vx_score_pages(gp, ctypes.byref(bad_table), FAKE, FAKE, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_topk_pages(gp, tp, FAKE, 0, 0, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # k = 0
+    assert L.vx_topk_pages(gp, tp, FAKE, 4, 2, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # mode 2
+    assert L.vx_centroid_update(gp, tp, None, None, FAKE, None, None, None, None, None) == vx.VX_ERR_INVALID_ARG
+    # append needs v_new for GQA
+    assert L.vx_centroid_update(gp, tp, FAKE, FAKE, FAKE, FAKE, None, None, None, None) == vx.VX_ERR_INVALID_ARG
+    # decode: workspace checked before launch (explicit split count: no device query needed)
+    assert L.vx_sparse_decode(gp, tp, FAKE, FAKE, FAKE, FAKE, 4, ctypes.c_float(0.0), 8, FAKE, None, None, 0,
+                              None, None) == vx.VX_ERR_WORKSPACE
+    need = L.vx_workspace_size(gp, 10, 4, 8)
+    assert need > 0
+    assert L.vx_sparse_decode(gp, tp, FAKE, FAKE, FAKE, FAKE, 4, ctypes.c_float(0.0), 8, FAKE, None, FAKE,
+                              need - 1, None, None) == vx.VX_ERR_WORKSPACE
+    assert L.vx_sparse_decode(gp, tp, FAKE, FAKE, FAKE, FAKE, 4, ctypes.c_float(float("nan")), 8, FAKE, None,
+                              FAKE, need, None, None) == vx.VX_ERR_INVALID_ARG
+
+
+def test_workspace_size_is_deterministic_and_monotone(L):
+    g = _geo()
+    gp = ctypes.byref(g)
+    a = L.vx_workspace_size(gp, 100, 16, 64)
+    assert a == L.vx_workspace_size(gp, 100, 16, 64)
+    assert L.vx_workspace_size(gp, 200, 16, 64) > a  # more pages -> larger score rows
+    assert L.vx_workspace_size(gp, 100, 32, 64) > a  # larger k
+    assert L.vx_workspace_size(gp, 100, 16, 128) > a  # more splits -> more partials
+    assert a % 256 == 0
+
+
+def test_status_strings(L):
+    assert L.vx_status_string(0) == b"VX_OK"
+    assert L.vx_status_string(3) == b"VX_ERR_WORKSPACE"
+    assert b"sm_100a" in L.vx_version()

@@ -1,0 +1,208 @@
+"""GPU parity: every step of the hot path through the C ABI against the fp64 oracle on
+the same seeded inputs, at sizes the oracle finishes in seconds that still span several
+tiles, splits and a ragged tail, plus the method's edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_cases import (check_attention, check_scores, err_word, geometry, gpu_centroids, gpu_decode, gpu_fused,
+                       gpu_scores, gpu_topk, host, recall, table, used_pages, workspace)
+from paged_block_sparse_kv_b200 import synth, vx
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny_config": (synth.SPECS["tiny_gqa4_d64"], 0),
+    "edges_1tok_fullpage_ragged": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=8, head_dim_qk=128,
+                                                     page_size=16, ctx=("list", [1, 16, 1000]), k=8), 11),
+    "g4_page32": (synth.custom_spec(batch=2, num_q_heads=8, num_kv_heads=2, head_dim_qk=128, page_size=32,
+                                    ctx=("list", [517, 64]), k=5), 12),
+    "g16_d64_page64": (synth.custom_spec(batch=2, num_q_heads=16, num_kv_heads=1, head_dim_qk=64, page_size=64,
+                                         ctx=("list", [300, 4097]), k=12), 13),
+    "g1_many_rows": (synth.custom_spec(batch=4, num_q_heads=8, num_kv_heads=8, head_dim_qk=128, page_size=16,
+                                       ctx=("uniform", 1, 3000), k=16), 14),
+    "k_exceeds_pages": (synth.custom_spec(batch=2, num_q_heads=4, num_kv_heads=2, head_dim_qk=128, page_size=16,
+                                          ctx=("list", [40, 90]), k=20), 15),
+    "qwen_shape_small_batch": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=8, head_dim_qk=128,
+                                                 page_size=16, ctx=("uniform", 4096, 9000), k=128, n_planted=8), 16),
+}
+
+_cache = {}
+
+
+def workload(name):
+    if name not in _cache:
+        spec, seed = CASES[name]
+        _cache[name] = synth.make(spec, seed, "cuda")
+    return _cache[name]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_step_by_step_parity(name):
+    w = workload(name)
+    h = host(w)
+    P = w.spec.page_size
+    err = err_word()
+    # a1: centroids, bit-exact with the oracle's correctly rounded mean
+    cen = gpu_centroids(w, err)
+    _, c16 = oracle.centroids(h["k"], h["ptr"], h["idx"], h["L"])
+    used = used_pages(h, P)
+    gc = synth.bits(cen)
+    assert np.array_equal(gc[used], c16[used]), "centroid mismatch"
+    # a2: scores, oracle scoring the same stored centroids
+    s = gpu_scores(w, cen, err=err)
+    s_orc = oracle.scores(h["q"], h["ptr"], h["idx"], h["L"], P, w.max_pages, w.spec.num_kv_heads,
+                          centroids_bf16=gc)
+    check_scores(s, s_orc, h["L"], P)
+    # a3: exact top-k, bit-exact with the oracle's stable sort on the GPU's own scores
+    sel = gpu_topk(w, s, err=err)
+    s_gpu = s.cpu().numpy().astype(np.float64)
+    sel_orc = oracle.topk_exact(s_gpu, h["L"], P, w.spec.k)
+    assert np.array_equal(sel.cpu().numpy(), sel_orc)
+    # a4: attention over the GPU's selection
+    out, lse = gpu_decode(w, sel, err=err)
+    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], sel=sel_orc)
+    check_attention(out, lse, o_orc, l_orc)
+    # fused entry = the three calls (same split plan -> identical bits)
+    out_f, lse_f, s_f, sel_f = gpu_fused(w, cen, err=err)
+    assert torch.equal(s_f, s) or np.array_equal(s_f.cpu().numpy(), s.cpu().numpy(), equal_nan=True)
+    assert torch.equal(sel_f, sel)
+    assert torch.equal(out_f, out) and torch.equal(lse_f, lse)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+
+
+@pytest.mark.parametrize("name", ["edges_1tok_fullpage_ragged", "g4_page32", "g16_d64_page64", "tiny_config"])
+def test_all_pages_equals_dense_attention(name):
+    w = workload(name)
+    h = host(w)
+    P = w.spec.page_size
+    n = (h["L"] + P - 1) // P
+    k = int(n.max())
+    sel = torch.full((w.batch, w.spec.num_kv_heads, k), -1, dtype=torch.int32)
+    for b in range(w.batch):
+        sel[b, :, :n[b]] = torch.arange(int(n[b]), dtype=torch.int32)
+    out, lse = gpu_decode(w, sel.cuda(), k=k)
+    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"])  # dense
+    check_attention(out, lse, o_orc, l_orc)
+
+
+@pytest.mark.parametrize("splits", [1, 3, 37, 0, 100000])
+def test_split_count_invariance(splits):
+    w = workload("g1_many_rows")
+    h = host(w)
+    cen = gpu_centroids(w)
+    sel = gpu_topk(w, gpu_scores(w, cen))
+    out, lse = gpu_decode(w, sel, num_splits=splits)
+    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], sel=sel.cpu().numpy())
+    check_attention(out, lse, o_orc, l_orc)
+
+
+def test_physical_page_permutation_is_bit_identical():
+    w = workload("qwen_shape_small_batch")
+    perm = torch.randperm(w.num_pool_pages, generator=torch.Generator().manual_seed(5)).cuda()
+    # page p moves to slot perm[p]
+    k2 = torch.empty_like(w.k_cache)
+    v2 = torch.empty_like(w.v_cache)
+    k2[perm] = w.k_cache
+    v2[perm] = w.v_cache
+    idx2 = perm[w.page_indices.long()].to(torch.int32)
+    w2 = synth.Workload(w.spec, w.seed, w.seq_lens, w.page_ptr, idx2, w.row_capacity, w.max_pages,
+                        w.num_pool_pages, k2, v2, w.q, w.planted)
+    a = gpu_fused(w, gpu_centroids(w))
+    b = gpu_fused(w2, gpu_centroids(w2))
+    for x, y in zip(a, b):
+        assert np.array_equal(x.cpu().numpy(), y.cpu().numpy(), equal_nan=True)
+
+
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "g1_many_rows", "g16_d64_page64"])
+def test_approx_topk_bit_exact_on_gpu_scores(name):
+    w = workload(name)
+    h = host(w)
+    s = gpu_scores(w, gpu_centroids(w))
+    s32 = s.cpu().numpy()
+    for seed in (0, 12345):
+        sel = gpu_topk(w, s, mode=1, seed=seed)
+        sel_orc = oracle.topk_approx(np.nan_to_num(s32, nan=0.0), h["L"], w.spec.page_size, w.spec.k, seed)
+        assert np.array_equal(sel.cpu().numpy(), sel_orc)
+    exact = oracle.topk_exact(s32.astype(np.float64), h["L"], w.spec.page_size, w.spec.k)
+    assert recall(sel.cpu().numpy(), exact) > 0.5
+
+
+def test_topk_ties_and_signed_zero():
+    # crafted rows: all-equal scores pick the lowest pages; -0.0 ties with +0.0
+    spec = synth.custom_spec(batch=2, num_q_heads=2, num_kv_heads=2, head_dim_qk=64, page_size=16,
+                             ctx=("list", [16 * 300, 16 * 40]), k=10)
+    w = synth.make(spec, 3, "cuda")
+    s = torch.zeros((2, 2, w.max_pages), dtype=torch.float32)
+    s[0, 1, ::2] = -0.0
+    s[1, 0, :] = torch.tensor(np.round(np.random.default_rng(0).standard_normal(w.max_pages)), dtype=torch.float32)
+    s[1, 1, 7] = 5.0
+    sel = gpu_topk(w, s.cuda())
+    sel_orc = oracle.topk_exact(s.numpy().astype(np.float64), w.seq_lens.cpu().numpy(), 16, 10)
+    assert np.array_equal(sel.cpu().numpy(), sel_orc)
+    assert sel[0, 0].tolist() == list(range(10))
+
+
+def test_append_steps_match_oracle():
+    # continuous batching: append one token per request per step, recompute tail centroids
+    spec = synth.custom_spec(batch=4, num_q_heads=8, num_kv_heads=4, head_dim_qk=128, page_size=16,
+                             ctx=("list", [15, 16, 33, 100]), k=4, steps=18)
+    w = synth.make(spec, 21, "cuda")
+    geo = geometry(w)
+    cen = gpu_centroids(w)
+    kc, vc = synth.bits(w.k_cache), synth.bits(w.v_cache)
+    ptr, idx = w.page_ptr.cpu().numpy(), w.page_indices.cpu().numpy()
+    err = err_word()
+    for s in range(spec.steps):
+        L = w.seq_lens_at(s)
+        vx.vx_centroid_update(geo, table(w, L), w.k_cache, cen, v_cache=w.v_cache, k_new=w.step_k_new[s],
+                              v_new=w.step_v_new[s], err=err)
+        kc, vc = oracle.append(kc, vc, ptr, idx, L.cpu().numpy(), synth.bits(w.step_k_new[s]),
+                               synth.bits(w.step_v_new[s]))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    Lf = w.seq_lens_at(spec.steps - 1).cpu().numpy()
+    hh = dict(L=Lf, ptr=ptr, idx=idx)
+    used = used_pages(hh, 16)
+    gk, gv = synth.bits(w.k_cache), synth.bits(w.v_cache)
+    assert np.array_equal(gk[used].view(np.int16), kc[used].view(np.int16))
+    assert np.array_equal(gv[used].view(np.int16), vc[used].view(np.int16))
+    _, c16 = oracle.centroids(kc, ptr, idx, Lf)
+    assert np.array_equal(synth.bits(cen)[used], c16[used])
+
+
+def test_bad_page_id_and_length_set_the_error_word():
+    w = synth.make(synth.custom_spec(batch=2, num_q_heads=4, num_kv_heads=2, head_dim_qk=128, page_size=16,
+                                     ctx=("list", [100, 200]), k=4), 9, "cuda")
+    cen = gpu_centroids(w)
+    bad_idx = w.page_indices.clone()
+    bad_idx[1] = w.num_pool_pages + 5  # out of the pool
+    wb = synth.Workload(w.spec, w.seed, w.seq_lens, w.page_ptr, bad_idx, w.row_capacity, w.max_pages,
+                        w.num_pool_pages, w.k_cache, w.v_cache, w.q, w.planted)
+    err = err_word()
+    out, lse, _, _ = gpu_fused(wb, cen, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & vx.VX_DATA_BAD_PAGE_ID
+    bad_len = w.seq_lens.clone()
+    bad_len[0] = w.max_pages * 16 + 1
+    err2 = err_word()
+    sc = torch.zeros((2, 2, w.max_pages), device="cuda")
+    vx.vx_score_pages(geometry(w), table(w, bad_len), w.q, cen, sc, err=err2)
+    torch.cuda.synchronize()
+    assert int(err2.item()) & vx.VX_DATA_BAD_SEQ_LEN
+    # the context is still usable
+    out_ok, _, _, _ = gpu_fused(w, cen)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out_ok.float()).all()
+
+
+def test_rope_unaware_score_dims():
+    w = workload("qwen_shape_small_batch")
+    h = host(w)
+    cen = gpu_centroids(w)
+    s = gpu_scores(w, cen, score_dims=64)
+    s_orc = oracle.scores(h["q"], h["ptr"], h["idx"], h["L"], 16, w.max_pages, 8, centroids_bf16=synth.bits(cen),
+                          score_dims=64)
+    check_scores(s, s_orc, h["L"], 16)
