@@ -1,0 +1,480 @@
+"""Benchmark: block top-k sparse attention decode over a paged KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--mode exact|approx]
+    python bench.py --impl reference ...     # the fp64 CPU oracle on the host cores
+
+A step is one decode step of one layer: score every page of every request from the
+cached centroids, select the top-k pages per (request, KV head), attend exactly over
+them (split-K + log-sum-exp merge); the continuous-batching workload first appends one
+token per request and updates the tail page's centroid.  `value` is query tokens/s per
+layer (batch / step time) summed over ranks.  Consecutive timed steps cycle through
+independent copies of the inputs (separate page pools, caches, centroids and queries)
+so that no step finds its working set in L2; steps are replayed from CUDA graphs and
+timed with CUDA events on the launching stream.
+
+Multi-GPU: every rank runs its own independent batch (weak scaling, no collective on
+the data path); timings are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-decode query tokens/s per layer; achieved HBM GB/s vs B200 peak"
+UNIT = "query tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+DEFAULT_CONFIG = "qwen3_1p7b_gqa_b32"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="vx", choices=["vx", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--mode", default="exact", choices=["exact", "approx"])
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (small profiling cases only)")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ peaks / clocks
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, enabled=True):
+        self.gpu_id, self.enabled, self.proc, self.lines = gpu_id, enabled, None, []
+
+    def __enter__(self):
+        if self.enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                     "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1].split()[0]))
+                mx.append(float(f[2].split()[0]))
+            except Exception:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ roofline bytes
+
+def step_bytes(w, sel, seq_lens, k):
+    """Algorithmic HBM bytes of one step: centroid reads + selected valid K/V tokens + q + out.
+
+    Returns (total, decode_part, centroid_part)."""
+    import numpy as np
+    s = w.spec
+    L = seq_lens.cpu().numpy().astype(np.int64)
+    P = s.page_size
+    n = (L + P - 1) // P
+    cen = int(n.sum()) * s.num_kv_heads * s.head_dim_qk * 2
+    sel_h = sel.cpu().numpy()
+    tok = 0
+    for b in range(len(L)):
+        rows = sel_h[b]
+        valid = rows[rows >= 0].astype(np.int64)
+        m = np.minimum(P, L[b] - valid * P)
+        tok += int(m.sum())  # summed over the KV heads
+    per_tok = s.head_dim_qk * 2 if s.mla_shared_kv else (s.head_dim_qk + s.head_dim_v) * 2
+    kv = tok * per_tok
+    qo = len(L) * s.num_q_heads * (s.head_dim_qk + s.head_dim_v) * 2
+    return cen + kv + qo, kv + qo, cen
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_vx(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from paged_block_sparse_kv_b200 import synth, vx
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    spec = synth.SPECS[args.config]
+    if args.batch:
+        spec = synth.Spec(**{**spec.__dict__, "batch": args.batch})
+    mode = 0 if args.mode == "exact" else 1
+    k = spec.k
+    B = spec.batch
+
+    def geom(w):
+        return vx.Geometry(w.batch, spec.num_q_heads, spec.num_kv_heads, spec.head_dim_qk, spec.head_dim_v,
+                           spec.page_size, spec.mla_shared_kv, w.num_pool_pages)
+
+    seed0 = 1000 * (list(synth.SPECS).index(args.config)) + 17 * rank
+
+    def buffers(w, geo):
+        out = torch.empty((B, spec.num_q_heads, spec.head_dim_v), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, spec.num_q_heads), dtype=torch.float32, device=dev)
+        scores = torch.empty((B, spec.num_kv_heads, w.max_pages), dtype=torch.float32, device=dev)
+        sel = torch.empty((B, spec.num_kv_heads, k), dtype=torch.int32, device=dev)
+        ws = torch.empty(vx.vx_workspace_size(geo, w.max_pages, k, args.splits), dtype=torch.uint8, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        return dict(out=out, lse=lse, scores=scores, sel=sel, ws=ws, err=err)
+
+    def rebuild_centroids(w, geo, tab):
+        cen = torch.zeros((w.num_pool_pages, spec.num_kv_heads, spec.head_dim_qk), dtype=torch.bfloat16, device=dev)
+        vx.vx_centroid_update(geo, tab, w.k_cache, cen, v_cache=w.v_cache)
+        return cen
+
+    def fused(c):
+        if c["append"]:
+            vx.vx_centroid_update(c["geo"], c["tab"], c["w"].k_cache, c["cen"], v_cache=c["w"].v_cache,
+                                  k_new=c["k_new"], v_new=c["v_new"], err=c["err"])
+        vx.vx_block_topk_decode(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"], k, c["out"],
+                                c["ws"], lse=c["lse"], mode=mode, seed=0, num_splits=args.splits,
+                                scores_out=c["scores"], sel_out=c["sel"], err=c["err"])
+
+    st = []
+    if spec.steps == 0:
+        # independent input copies, rotated so no step finds its inputs in L2
+        w = synth.make(spec, seed0, dev)
+        geo = geom(w)
+        tab = vx.PageTable(w.page_ptr, w.page_indices, w.seq_lens, w.max_pages)
+        st.append(dict(w=w, geo=geo, tab=tab, cen=rebuild_centroids(w, geo, tab), q=w.q, append=False,
+                       seq_lens=w.seq_lens, **buffers(w, geo)))
+        fused(st[0])
+        torch.cuda.synchronize()
+        total0 = step_bytes(w, st[0]["sel"], w.seq_lens, k)[0]
+        for i in range(1, max(2, math.ceil(3 * L2_BYTES / max(total0, 1)))):
+            w = synth.make(spec, seed0 + i, dev)
+            geo = geom(w)
+            tab = vx.PageTable(w.page_ptr, w.page_indices, w.seq_lens, w.max_pages)
+            st.append(dict(w=w, geo=geo, tab=tab, cen=rebuild_centroids(w, geo, tab), q=w.q, append=False,
+                           seq_lens=w.seq_lens, **buffers(w, geo)))
+        launches_per_step = 4
+        l2_note = "inputs rotate over {n} independent copies, {mb:.0f} MB between reuses (> 3x L2)"
+    else:
+        # continuous batching: one workload, `steps` consecutive decode steps, each appending
+        # one token per request before it decodes (replays rewrite the same slots)
+        w = synth.make(spec, seed0, dev)
+        geo = geom(w)
+        lens = torch.stack([w.seq_lens_at(s_) for s_ in range(spec.steps)]).contiguous()
+        cen = rebuild_centroids(w, geo, vx.PageTable(w.page_ptr, w.page_indices, w.seq_lens, w.max_pages))
+        shared = buffers(w, geo)
+        for s_ in range(spec.steps):
+            tab = vx.PageTable(w.page_ptr, w.page_indices, lens[s_], w.max_pages)
+            ctx = dict(w=w, geo=geo, tab=tab, cen=cen, q=w.step_q[s_], append=True, k_new=w.step_k_new[s_],
+                       v_new=w.step_v_new[s_], seq_lens=lens[s_], **shared)
+            ctx["sel"] = torch.empty_like(shared["sel"])
+            st.append(ctx)
+        launches_per_step = 5
+        l2_note = "{n} consecutive appending decode steps over one {mb:.0f} MB-per-step working set (> L2)"
+    for c in st:
+        fused(c)
+    torch.cuda.synchronize()
+    per_copy = [step_bytes(c["w"], c["sel"], c["seq_lens"], k) for c in st]
+
+    stream = torch.cuda.Stream(device=dev)
+    def capture(n_steps, start, fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n_steps):
+                    fn(st[(start + i) % len(st)])
+        return g
+
+    def timed_replay(fn, steps, warmup, chunk=500):
+        # warm-up (eager) then graphs of `chunk` steps; exactly `steps` timed steps
+        with torch.cuda.stream(stream):
+            for i in range(warmup):
+                fn(st[i % len(st)])
+        torch.cuda.synchronize()
+        c = min(chunk, steps)
+        c -= c % len(st) if c >= len(st) else 0
+        c = max(c, 1)
+        full, rem = divmod(steps, c)
+        g_full = capture(c, 0, fn)
+        g_rem = capture(rem, 0, fn) if rem else None
+        torch.cuda.synchronize()
+        g_full.replay()  # one untimed replay primes the graph
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(full):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms, (g_full, c)
+
+    gpu_id = _gpu_id(local_rank)
+    with ClockSampler(gpu_id, enabled=not args.no_clocks and rank == 0) as clk:
+        ms_total, (g_full, chunk) = timed_replay(fused, args.steps, args.warmup)
+        # keep the GPU in the same steady state for >= 1 s so the sampler sees it
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            with torch.cuda.stream(stream):
+                g_full.replay()
+            torch.cuda.synchronize()
+    clocks = clk.summary()
+
+    ms_step = ms_total / args.steps
+    mean_bytes = sum(p[0] for p in per_copy) / len(per_copy)
+    tok_s = B / (ms_step * 1e-3) * world
+    peak, peak_kind = peaks()
+    step_gbs = mean_bytes / (ms_step * 1e-3) / 1e9
+
+    # dominant kernel: the sparse decode call (gather-attention kernel + its merge), timed alone
+    def decode_only(c):
+        vx.vx_sparse_decode(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["sel"], k, c["out"],
+                            c["ws"], lse=c["lse"], num_splits=args.splits, err=c["err"])
+    dec_steps = max(len(st), min(args.steps, 1000))
+    ms_dec, _ = timed_replay(decode_only, dec_steps, 3)
+    ms_dec_launch = ms_dec / dec_steps
+    dec_bytes = sum(p[1] for p in per_copy) / len(per_copy)
+    dec_gbs = dec_bytes / (ms_dec_launch * 1e-3) / 1e9
+
+    # end to end through the public call with host buffers: per step H2D of the query and
+    # page table from pinned memory, the fused call, D2H of the outputs
+    c = st[0]
+    w = c["w"]
+    h_q = c["q"].cpu().pin_memory()
+    h_ptr, h_idx, h_len = (w.page_ptr.cpu().pin_memory(), w.page_indices.cpu().pin_memory(),
+                           c["seq_lens"].cpu().pin_memory())
+    h_out = torch.empty(c["out"].shape, dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty(c["lse"].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_ptr, h_idx, h_len))
+    d2h = h_out.numel() * 2 + h_lse.numel() * 4
+    e2e_steps = max(1, args.e2e_steps)
+    with torch.cuda.stream(stream):
+        for it in range(3 + e2e_steps):
+            if it == 3:
+                torch.cuda.synchronize()
+                if world > 1:
+                    dist.barrier()
+                ev0 = torch.cuda.Event(enable_timing=True)
+                ev0.record(stream)
+            c["q"].copy_(h_q, non_blocking=True)
+            w.page_ptr.copy_(h_ptr, non_blocking=True)
+            w.page_indices.copy_(h_idx, non_blocking=True)
+            c["seq_lens"].copy_(h_len, non_blocking=True)
+            fused(c)
+            h_out.copy_(c["out"], non_blocking=True)
+            h_lse.copy_(c["lse"], non_blocking=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = ev0.elapsed_time(ev1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    errs = [int(c["err"].item()) for c in st]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(st[0]["w"], st[0]["cen"], k, st[0]["seq_lens"], st[0]["q"])
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(tok_s, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.config + (f" (batch overridden to {B})" if args.batch else ""), "batch": B, "num_q_heads": spec.num_q_heads,
+                       "num_kv_heads": spec.num_kv_heads, "head_dim_qk": spec.head_dim_qk,
+                       "head_dim_v": spec.head_dim_v, "page_size": spec.page_size, "k_pages": k,
+                       "context": list(spec.ctx), "topk_mode": args.mode, "splits": args.splits or "planned",
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": l2_note.format(n=len(st), mb=mean_bytes * max(1, len(st) - 1) / 1e6)},
+            "hbm": {"roofline_bytes_per_step": int(mean_bytes), "achieved_gbs": round(step_gbs, 1),
+                    "peak_gbs": peak, "frac": round(step_gbs / peak, 4), "peak_kind": peak_kind,
+                    "centroid_bytes": int(sum(p[2] for p in per_copy) / len(per_copy))},
+            "roofline": {"bound": "hbm", "kernel": "sparse decode (gather-attention + merge)",
+                         "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(dec_gbs / peak, 4), "traffic": None,
+                         "bytes_per_launch": int(dec_bytes), "us_per_launch": round(ms_dec_launch * 1e3, 3),
+                         "peak_kind": peak_kind},
+            "e2e": {"value": round(B / (ms_e2e * 1e-3) * world, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "device_errors": errs,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _gpu_id(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",")]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+
+def cpu_baseline(w, cen, k, seq_lens, q, budget_s=12.0):
+    """The oracle, as it stands, on the host cores over a bounded sample of the workload:
+    the first requests of one step, repeated for about `budget_s` seconds."""
+    import torch
+
+    import oracle
+    from paged_block_sparse_kv_b200 import synth
+    reqs = list(range(min(4, w.batch)))
+    h = synth.host_subset(w, reqs, seq_lens=seq_lens)
+    cen_h = synth.bits(cen[torch.as_tensor(h["phys"], dtype=torch.int64, device=cen.device)])
+    P = w.spec.page_size
+    maxp = int(((h["seq_lens"] + P - 1) // P).max())
+    args = (synth.bits(q[:len(reqs)]), h["k_cache"], h["v_cache"], cen_h, h["page_ptr"], h["page_indices"],
+            h["seq_lens"], maxp, k)
+    kw = dict(mla_shared_kv=w.spec.mla_shared_kv, head_dim_v=w.spec.head_dim_v)
+    t0 = time.perf_counter()
+    oracle.decode_step(*args, **kw)
+    one = time.perf_counter() - t0
+    reps = max(1, min(50, int(budget_s / max(one, 1e-6))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.decode_step(*args, **kw)
+    dt = time.perf_counter() - t0
+    return {"value": round(len(reqs) * reps / dt, 3), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(reqs)} of {w.batch} requests x {reps} decode steps (score + exact top-k + "
+                      f"attention, fp64), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world, budget_s=150.0):
+    """The fp64 oracle, as it stands, timed on the host cores: each step is a bounded sample
+    of the workload (2 requests; fewer KV heads when K + W steps of that would not fit in
+    about `budget_s` seconds)."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from paged_block_sparse_kv_b200 import synth
+    spec = synth.SPECS[args.config]
+    w = synth.make(synth.Spec(**{**spec.__dict__, "steps": 0}), 1000 * list(synth.SPECS).index(args.config),
+                   "cpu", batch=min(spec.batch, 2))
+    h = synth.host_subset(w, list(range(w.batch)))
+    _, cen16 = oracle.centroids(h["k_cache"], h["page_ptr"], h["page_indices"], h["seq_lens"])
+    maxp = int(((h["seq_lens"] + spec.page_size - 1) // spec.page_size).max())
+    q = synth.bits(w.q)
+    G = spec.num_q_heads // spec.num_kv_heads
+
+    def call(hk):
+        v = None if h["v_cache"] is None else np.ascontiguousarray(h["v_cache"][:, :hk])
+        return oracle.decode_step(np.ascontiguousarray(q[:, :hk * G]), np.ascontiguousarray(h["k_cache"][:, :hk]), v,
+                                  np.ascontiguousarray(cen16[:, :hk]), h["page_ptr"], h["page_indices"],
+                                  h["seq_lens"], maxp, spec.k, mla_shared_kv=spec.mla_shared_kv,
+                                  head_dim_v=spec.head_dim_v)
+
+    t0 = time.perf_counter()
+    call(spec.num_kv_heads)
+    one = time.perf_counter() - t0
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    hk = spec.num_kv_heads if one <= per_step else max(1, int(spec.num_kv_heads * per_step / one))
+    for _ in range(args.warmup):
+        call(hk)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        call(hk)
+    dt = time.perf_counter() - t0
+    req_per_step = w.batch * hk / spec.num_kv_heads
+    value = req_per_step * args.steps / dt
+    sample = (f"{w.batch} of {spec.batch} requests, {hk} of {spec.num_kv_heads} KV heads per step "
+              f"(score + exact top-k + attention, fp64)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.config, "k_pages": spec.k, "sample": sample},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_vx(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -33,11 +33,6 @@ struct TileMeta {
     int32_t nvalid;
 };
 
-struct Resolved {
-    int32_t row, z, y, nvalid;  // row, tensor-map page-head index, token offset, valid tokens
-    bool valid;
-};
-
 __device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u, int64_t u_end) {
     Resolved rs{0, 0, 0, 0, false};
     if (u >= u_end) return rs;

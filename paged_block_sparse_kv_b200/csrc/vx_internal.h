@@ -76,6 +76,13 @@ struct DecodeArgs {
     float scale_log2;         // sm_scale * log2(e)
 };
 
+// One decode work unit (a 16-token tile of a selected page) after its metadata has been
+// looked up: row, tensor-map page(-head) index, token offset in the page, valid tokens.
+struct Resolved {
+    int32_t row, z, y, nvalid;
+    bool valid;
+};
+
 // ------------------------------------------------------------------ launches
 cudaError_t launch_centroid(const CentroidArgs &a, bool append, cudaStream_t s);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s, bool pdl);

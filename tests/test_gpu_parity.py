@@ -26,7 +26,15 @@ CASES = {
                                           ctx=("list", [40, 90]), k=20), 15),
     "qwen_shape_small_batch": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=8, head_dim_qk=128,
                                                  page_size=16, ctx=("uniform", 4096, 9000), k=128, n_planted=8), 16),
+    "mla_16heads": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
+                                      page_size=64, mla_shared_kv=True, ctx=("list", [700, 2000, 64]), k=6), 17),
+    "mla_5heads_ragged": (synth.custom_spec(batch=2, num_q_heads=5, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
+                                            page_size=64, mla_shared_kv=True, ctx=("list", [1, 4000]), k=9), 18),
 }
+
+
+def attend_kw(w):
+    return dict(mla_shared_kv=w.spec.mla_shared_kv, head_dim_v=w.spec.head_dim_v)
 
 _cache = {}
 
@@ -62,7 +70,7 @@ def test_step_by_step_parity(name):
     assert np.array_equal(sel.cpu().numpy(), sel_orc)
     # a4: attention over the GPU's selection
     out, lse = gpu_decode(w, sel, err=err)
-    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], sel=sel_orc)
+    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], sel=sel_orc, **attend_kw(w))
     check_attention(out, lse, o_orc, l_orc)
     # fused entry = the three calls (same split plan -> identical bits)
     out_f, lse_f, s_f, sel_f = gpu_fused(w, cen, err=err)
@@ -73,7 +81,8 @@ def test_step_by_step_parity(name):
     assert int(err.item()) == 0
 
 
-@pytest.mark.parametrize("name", ["edges_1tok_fullpage_ragged", "g4_page32", "g16_d64_page64", "tiny_config"])
+@pytest.mark.parametrize("name", ["edges_1tok_fullpage_ragged", "g4_page32", "g16_d64_page64", "tiny_config",
+                                  "mla_16heads"])
 def test_all_pages_equals_dense_attention(name):
     w = workload(name)
     h = host(w)
@@ -84,18 +93,20 @@ def test_all_pages_equals_dense_attention(name):
     for b in range(w.batch):
         sel[b, :, :n[b]] = torch.arange(int(n[b]), dtype=torch.int32)
     out, lse = gpu_decode(w, sel.cuda(), k=k)
-    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"])  # dense
+    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], **attend_kw(w))  # dense
     check_attention(out, lse, o_orc, l_orc)
 
 
+@pytest.mark.parametrize("name", ["g1_many_rows", "mla_16heads"])
 @pytest.mark.parametrize("splits", [1, 3, 37, 0, 100000])
-def test_split_count_invariance(splits):
-    w = workload("g1_many_rows")
+def test_split_count_invariance(name, splits):
+    w = workload(name)
     h = host(w)
     cen = gpu_centroids(w)
     sel = gpu_topk(w, gpu_scores(w, cen))
     out, lse = gpu_decode(w, sel, num_splits=splits)
-    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], sel=sel.cpu().numpy())
+    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], sel=sel.cpu().numpy(),
+                                 **attend_kw(w))
     check_attention(out, lse, o_orc, l_orc)
 
 
@@ -113,10 +124,11 @@ def test_physical_page_permutation_is_bit_identical():
     a = gpu_fused(w, gpu_centroids(w))
     b = gpu_fused(w2, gpu_centroids(w2))
     for x, y in zip(a, b):
-        assert np.array_equal(x.cpu().numpy(), y.cpu().numpy(), equal_nan=True)
+        assert torch.equal(x.view(torch.int16) if x.dtype == torch.bfloat16 else x.view(torch.int32),
+                           y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32))
 
 
-@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "g1_many_rows", "g16_d64_page64"])
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "g1_many_rows", "g16_d64_page64", "mla_16heads"])
 def test_approx_topk_bit_exact_on_gpu_scores(name):
     w = workload(name)
     h = host(w)
