@@ -95,9 +95,9 @@ typedef struct {
 
 /*
  * Cache stage: key centroid of a page = mean of the keys of its valid tokens, per KV
- * head, stored as bf16 (the cache's element type) after one round-to-nearest-even of
- * the fp32 mean (paper note, 系统设计 1: the cache stage keeps a per-block key centroid
- * that does not depend on the query).
+ * head, stored as bf16 (the cache's element type): the exact mean (fp64 sum of the bf16
+ * keys, one fp64 division) rounded once to nearest-even (paper note, 系统设计 1: the
+ * cache stage keeps a per-block key centroid that does not depend on the query).
  *   k_new == NULL: rebuild.  Recompute the centroid of every page of every request
  *       holding a position >= first_pos[b] (first_pos NULL: every page).  Use after a
  *       prefill or a bulk load.  v_cache, v_new unused.
@@ -153,8 +153,9 @@ vx_status vx_topk_pages(const vx_geometry *geo, const vx_page_table *table, cons
  * whose partial (o, max, sum) are merged with the log-sum-exp rule.
  *   sm_scale <= 0 means 1 / sqrt(head_dim_qk).  num_splits 0 = planned from the SM count.
  *   lse may be NULL.  A request with no attended token gets out = 0, lse = -inf.
- * ws: device workspace of at least vx_workspace_size(geo, max_pages, k, num_splits)
- * bytes (the split partials).
+ * ws: device workspace for the split partials; vx_workspace_size(geo, max_pages, k,
+ * num_splits) bytes are always enough (that size also covers the fused call's scores
+ * and selection, which this call does not use).
  */
 vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, const void *q,
                            const void *k_cache, const void *v_cache, const int32_t *sel, int32_t k,

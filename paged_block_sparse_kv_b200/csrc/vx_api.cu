@@ -168,6 +168,9 @@ WsLayout ws_layout(const vx_geometry *g, int32_t max_pages, int32_t k, const Pla
     return l;
 }
 
+// bytes vx_sparse_decode uses: the split partials only (they sit at the start of the layout)
+size_t decode_ws_bytes(const WsLayout &l) { return l.scores; }
+
 // ------------------------------------------------------------------ TMA descriptors
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -428,8 +431,8 @@ vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, c
     VX_TRY(plan(geo, k, num_splits, &p));
     const WsLayout l = ws_layout(geo, table->max_pages, k, p);
     if (!ws || !al16(ws)) return fail(VX_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
-    if (ws_bytes < l.total)
-        return fail(VX_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, l.total);
+    if (ws_bytes < decode_ws_bytes(l))
+        return fail(VX_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, decode_ws_bytes(l));
     return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, ws, out, lse, err,
                      static_cast<cudaStream_t>(stream), false);
 }

@@ -102,8 +102,13 @@ def test_bad_pointers_and_sizes(L):
                               None, None) == vx.VX_ERR_WORKSPACE
     need = L.vx_workspace_size(gp, 10, 4, 8)
     assert need > 0
+    # the decode call needs only its split partials: (rows + splits) * G * (Dv + 2) floats, 256-aligned
+    rows, G = 2 * 8, 2
+    partial = -(-(rows + 8) * G * 128 * 4 // 256) * 256 + -(-(rows + 8) * G * 2 * 4 // 256) * 256
+    assert partial < need
     assert L.vx_sparse_decode(gp, tp, FAKE, FAKE, FAKE, FAKE, 4, ctypes.c_float(0.0), 8, FAKE, None, FAKE,
-                              need - 1, None, None) == vx.VX_ERR_WORKSPACE
+                              partial - 1, None, None) == vx.VX_ERR_WORKSPACE
+    assert b"needed" in L.vx_last_error()
     assert L.vx_sparse_decode(gp, tp, FAKE, FAKE, FAKE, FAKE, 4, ctypes.c_float(float("nan")), 8, FAKE, None,
                               FAKE, need, None, None) == vx.VX_ERR_INVALID_ARG
 
