@@ -178,6 +178,35 @@ vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *tabl
                                int32_t *err, void *stream);
 
 /*
+ * vx_sparse_decode without a caller workspace, for callers that cannot allocate device
+ * memory.  This entry point has no counterpart in the paper; it exists for integration.
+ * Who needs it: an inference engine that gives all free HBM to its KV-cache pool at
+ * start-up and allows no later cudaMalloc, a plugin interface that hands over tensors but
+ * no workspace, or a caller that must avoid the device synchronisation cudaMalloc and
+ * cudaFree can cause.
+ * What it does: exactly vx_sparse_decode (same arguments minus ws / ws_bytes, same
+ * results), with the split partials kept in one array of VX_NOALLOC_SCRATCH_BYTES that
+ * the library holds in device memory, once per GPU, until the process exits.  It
+ * allocates nothing and calls no allocating routine.
+ *   - Limit: a problem whose split partials need more than VX_NOALLOC_SCRATCH_BYTES
+ *     ((rows + splits) * G * (head_dim_v + 2) * 4 bytes, rows = batch * num_kv_heads)
+ *     is rejected with VX_ERR_WORKSPACE and a message; pass fewer splits or use
+ *     vx_sparse_decode with your own workspace.
+ *   - Set-up: the first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current).  Make that first call on a
+ *     device before any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps whatever the last
+ *     call left in it; nothing in it has to start at zero (a call writes each partial
+ *     before reading it).  Calls that overlap on the GPU (two streams, or two host
+ *     threads, at once) race on the array: order them on one stream.
+ */
+#define VX_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+vx_status vx_sparse_decode_noalloc(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                                   const void *k_cache, const void *v_cache, const int32_t *sel,
+                                   int32_t k, float sm_scale, int32_t num_splits, void *out,
+                                   float *lse, int32_t *err, void *stream);
+
+/*
  * Workspace bytes that vx_sparse_decode and vx_block_topk_decode need for this geometry,
  * row bound, k and split count (0 = the planned count); 0 when the arguments are
  * invalid (see vx_last_error).  Deterministic: the same inputs give the same size.

@@ -306,6 +306,26 @@ vx_status check_k_mode(int32_t k, int32_t mode) {
 
 }  // namespace
 
+namespace vx {
+
+vx_status decode_partial_bytes(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits,
+                               size_t *bytes) {
+    VX_TRY(check_geometry(geo));
+    VX_TRY(check_max_pages(geo, max_pages));
+    VX_TRY(check_k_mode(k, 0));
+    Plan p;
+    VX_TRY(plan(geo, k, num_splits, &p));
+    *bytes = decode_ws_bytes(ws_layout(geo, max_pages, k, p));
+    return VX_OK;
+}
+
+vx_status set_error(vx_status s, const char *msg) {
+    g_last_error = msg;
+    return s;
+}
+
+}  // namespace vx
+
 // ==================================================================== C ABI
 
 extern "C" {

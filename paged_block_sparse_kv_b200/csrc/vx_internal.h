@@ -93,6 +93,13 @@ cudaError_t launch_decode_mla(const DecodeArgs &a, const CUtensorMap &tmK, int g
                               bool pdl);
 cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl);
 
+// Host helpers of the C ABI layer (vx_api.cu).
+// Bytes of split partials vx_sparse_decode needs for this problem (validates the geometry).
+vx_status decode_partial_bytes(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits,
+                               size_t *bytes);
+// Set the message vx_last_error() returns on this host thread; returns s.
+vx_status set_error(vx_status s, const char *msg);
+
 // Launch with programmatic dependent launch enabled when `pdl` (the kernel must call
 // pdl_wait() before reading what the previous kernel on the stream wrote).
 template <typename... KArgs, typename... Args>

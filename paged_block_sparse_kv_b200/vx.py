@@ -22,7 +22,7 @@ VX_DATA_BAD_PAGE_ID, VX_DATA_BAD_SEQ_LEN, VX_DATA_BAD_SELECTION, VX_DATA_TIMEOUT
 
 # every symbol include/vx.h declares
 EXPORTS = ["vx_centroid_update", "vx_score_pages", "vx_topk_pages", "vx_sparse_decode",
-           "vx_block_topk_decode", "vx_workspace_size", "vx_planned_splits", "vx_status_string",
+           "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_workspace_size", "vx_planned_splits", "vx_status_string",
            "vx_last_error", "vx_version"]
 
 
@@ -60,6 +60,7 @@ def lib():
         L.vx_score_pages.argtypes = [G, T, p, p, i32, p, p, p]
         L.vx_topk_pages.argtypes = [G, T, p, i32, i32, u64, p, p, p]
         L.vx_sparse_decode.argtypes = [G, T, p, p, p, p, i32, f32, i32, p, p, p, sz, p, p]
+        L.vx_sparse_decode_noalloc.argtypes = [G, T, p, p, p, p, i32, f32, i32, p, p, p, p]
         L.vx_block_topk_decode.argtypes = [G, T, p, p, p, p, i32, i32, u64, f32, i32, i32, p, p, p, p, p, sz,
                                            p, p]
         L.vx_workspace_size.argtypes = [G, i32, i32, i32]
@@ -71,7 +72,7 @@ def lib():
         L.vx_last_error.restype = ctypes.c_char_p
         L.vx_version.restype = ctypes.c_char_p
         for name in ("vx_centroid_update", "vx_score_pages", "vx_topk_pages", "vx_sparse_decode",
-                     "vx_block_topk_decode"):
+                     "vx_sparse_decode_noalloc", "vx_block_topk_decode"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -178,6 +179,17 @@ def vx_sparse_decode(geo: Geometry, table: PageTable, q, k_cache, v_cache, sel, 
                                _ptr(k_cache, torch.bfloat16), _ptr(v_cache, torch.bfloat16), _ptr(sel, torch.int32),
                                k, float(sm_scale), num_splits, _ptr(out, torch.bfloat16), _ptr(lse, torch.float32),
                                _ptr(ws), ws.numel() * ws.element_size(), _ptr(err, torch.int32), _stream(stream)))
+
+
+def vx_sparse_decode_noalloc(geo: Geometry, table: PageTable, q, k_cache, v_cache, sel, k: int, out, lse=None,
+                             sm_scale=0.0, num_splits=0, err=None, stream=None):
+    """vx_sparse_decode for callers that cannot allocate device memory: the split partials
+    live in a fixed scratch array inside the library (see include/vx.h)."""
+    _ok(lib().vx_sparse_decode_noalloc(ctypes.byref(geo.c()), ctypes.byref(table.c()), _ptr(q, torch.bfloat16),
+                                       _ptr(k_cache, torch.bfloat16), _ptr(v_cache, torch.bfloat16),
+                                       _ptr(sel, torch.int32), k, float(sm_scale), num_splits,
+                                       _ptr(out, torch.bfloat16), _ptr(lse, torch.float32), _ptr(err, torch.int32),
+                                       _stream(stream)))
 
 
 def vx_block_topk_decode(geo: Geometry, table: PageTable, q, k_cache, v_cache, centroids, k: int, out, ws,

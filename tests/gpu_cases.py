@@ -145,3 +145,9 @@ def recall(sel_a, sel_b):
         if ys:
             vals.append(len(ys & set(int(v) for v in x if v >= 0)) / len(ys))
     return float(np.mean(vals))
+
+
+def check_attention_pair(out, lse, out_ref, lse_ref):
+    """Two GPU results of the same attention, compared with the parity tolerance."""
+    return check_attention(out, lse, out_ref.float().cpu().numpy().astype(np.float64),
+                           lse_ref.cpu().numpy().astype(np.float64))
