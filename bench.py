@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--breakdown", action="store_true",
+                    help="also time the score, top-k and decode calls separately (CUDA events, graphs)")
     return ap.parse_args()
 
 
@@ -319,6 +321,27 @@ def run_vx(args, rank, world, local_rank):
     dec_bytes = sum(p[1] for p in per_copy) / len(per_copy)
     dec_gbs = dec_bytes / (ms_dec_launch * 1e-3) / 1e9
 
+    breakdown = None
+    if args.breakdown:
+        def score_only(c):
+            vx.vx_score_pages(c["geo"], c["tab"], c["q"], c["cen"], c["scores"], err=c["err"])
+
+        def topk_only(c):
+            vx.vx_topk_pages(c["geo"], c["tab"], c["scores"], k, c["sel"], mode=mode, seed=0, err=c["err"])
+
+        nb = max(len(st), min(args.steps, 1000))
+        breakdown = {}
+        for name, fn in (("score", score_only), ("topk", topk_only), ("decode_merge", decode_only)):
+            ms_b, _ = timed_replay(fn, nb, 3)
+            breakdown[name + "_us"] = round(ms_b / nb * 1e3, 3)
+        if spec.steps:
+            def append_only(c):
+                vx.vx_centroid_update(c["geo"], c["tab"], c["w"].k_cache, c["cen"], v_cache=c["w"].v_cache,
+                                      k_new=c["k_new"], v_new=c["v_new"], err=c["err"])
+            ms_b, _ = timed_replay(append_only, nb, 3)
+            breakdown["append_us"] = round(ms_b / nb * 1e3, 3)
+        breakdown["step_us"] = round(ms_step * 1e3, 3)
+
     # end to end through the public call with host buffers: per step H2D of the query and
     # page table from pinned memory, the fused call, D2H of the outputs
     c = st[0]
@@ -385,6 +408,7 @@ def run_vx(args, rank, world, local_rank):
             "e2e": {"value": round(B / (ms_e2e * 1e-3) * world, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
             "gpu_launches": launches_per_step * args.steps,
+            "breakdown": breakdown,
             "clocks": clocks,
             "device_errors": errs,
         }

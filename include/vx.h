@@ -76,12 +76,12 @@ typedef enum {
 #define VX_DATA_TIMEOUT 8u       /* a bounded wait inside a kernel ran out */
 
 typedef struct {
-    int32_t batch;         /* B >= 1 */
+    int32_t batch;         /* 1 <= B <= 4096 */
     int32_t num_q_heads;   /* Hq, a multiple of num_kv_heads */
-    int32_t num_kv_heads;  /* Hkv */
+    int32_t num_kv_heads;  /* Hkv: GQA a power of two <= 16, MLA 1 */
     int32_t head_dim_qk;   /* key / score dim: 64 or 128 (GQA), 576 (MLA latent+rope) */
     int32_t head_dim_v;    /* value dim: = head_dim_qk (GQA), 512 (MLA) */
-    int32_t page_size;     /* P tokens per page: 16, 32 or 64 (MLA: 64) */
+    int32_t page_size;     /* P tokens per page: 16, 32 or 64 (MLA: 32 or 64) */
     int32_t mla_shared_kv; /* 1: V = first head_dim_v dims of the K row; v_cache unused */
     int64_t num_pool_pages;
 } vx_geometry;

@@ -343,49 +343,82 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     for (int64_t r = flushed_to + 1; r <= row_last; ++r) write_empty(r);
 }
 
-// Merge: one warp per (row, query head of the group).
+// Merge: one warp per (row, query head of the group, slice of MERGE_DIMS output dims).
+// The row's partials are those of the chunks c_lo..c_hi that touch it (slot row + c).
+// Lanes first read every partial's (max, sum) in parallel to form the common max and the
+// total; the weighted outputs are then accumulated MERGE_UNROLL partials at a time, each
+// lane owning MERGE_DIMS/32 dims of the slice.
+constexpr int MERGE_UNROLL = 4;
+constexpr int MERGE_DIMS = 128;
+
 template <int DV>
 __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     pdl_wait();
+    constexpr int SLICE = DV < MERGE_DIMS ? DV : MERGE_DIMS;
+    constexpr int NSLICE = DV / SLICE;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t item = (int64_t)blockIdx.x * 8 + warp;
     const int64_t rows = (int64_t)a.B * a.Hkv;
-    if (item >= rows * a.G) return;
-    const int64_t r = item / a.G;
-    const int g = static_cast<int>(item % a.G);
+    if (item >= rows * a.G * NSLICE) return;
+    const int slice = static_cast<int>(item % NSLICE);
+    const int64_t rg = item / NSLICE;
+    const int64_t r = rg / a.G;
+    const int g = static_cast<int>(rg % a.G);
     const int64_t c_lo = chunk_of(r * a.units_per_row, a.units, a.chunks);
     const int64_t c_hi = chunk_of((r + 1) * a.units_per_row - 1, a.units, a.chunks);
+    const int np = static_cast<int>(c_hi - c_lo + 1);
+    const float *ml0 = a.ml_part + ((r + c_lo) * a.G + g) * 2;                    // partial i at + i*G*2
+    const float *o0 = a.o_part + ((r + c_lo) * a.G + g) * DV + slice * SLICE;      // partial i at + i*G*DV
+    // common max and total over all partials (lane i handles partials i, i + 32, ...)
     float M = -INFINITY;
-    for (int64_t cc = c_lo; cc <= c_hi; ++cc) M = fmaxf(M, a.ml_part[((r + cc) * a.G + g) * 2]);
-    constexpr int PER = DV / 32;  // dims per lane
+    for (int i = lane; i < np; i += 32) M = fmaxf(M, ml0[(int64_t)i * a.G * 2]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+    float lsum = 0.f;
+    if (M != -INFINITY)
+        for (int i = lane; i < np; i += 32) {
+            const float m = ml0[(int64_t)i * a.G * 2];
+            if (m != -INFINITY) lsum += exp2f(m - M) * ml0[(int64_t)i * a.G * 2 + 1];
+        }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(FULL, lsum, off);
+
+    constexpr int PER = SLICE / 32;  // dims per lane
     float o[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) o[i] = 0.f;
-    float lsum = 0.f;
     if (M != -INFINITY) {
-        for (int64_t cc = c_lo; cc <= c_hi; ++cc) {
-            const float *ml = a.ml_part + ((r + cc) * a.G + g) * 2;
-            const float m = ml[0];
-            if (m == -INFINITY) continue;
-            const float w = exp2f(m - M);
-            lsum += w * ml[1];
-            const float *op = a.o_part + ((r + cc) * a.G + g) * DV + lane * PER;
+        for (int i0 = 0; i0 < np; i0 += MERGE_UNROLL) {
+            float w[MERGE_UNROLL];
+            float2 v[MERGE_UNROLL][PER / 2];
 #pragma unroll
-            for (int i = 0; i < PER; i += 2) {
-                const float2 v = *reinterpret_cast<const float2 *>(op + i);
-                o[i] += w * v.x;
-                o[i + 1] += w * v.y;
+            for (int u = 0; u < MERGE_UNROLL; ++u) {
+                const int i = i0 + u;
+                const float m = i < np ? ml0[(int64_t)i * a.G * 2] : -INFINITY;
+                w[u] = m == -INFINITY ? 0.f : exp2f(m - M);
+                const float *op = o0 + (int64_t)i * a.G * DV + lane * PER;
+#pragma unroll
+                for (int d = 0; d < PER / 2; ++d)
+                    v[u][d] = w[u] != 0.f ? *reinterpret_cast<const float2 *>(op + 2 * d) : make_float2(0.f, 0.f);
             }
+#pragma unroll
+            for (int u = 0; u < MERGE_UNROLL; ++u)
+#pragma unroll
+                for (int d = 0; d < PER / 2; ++d) {
+                    o[2 * d] += w[u] * v[u][d].x;
+                    o[2 * d + 1] += w[u] * v[u][d].y;
+                }
         }
     }
     const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);
     const size_t head = (size_t)b * a.Hq + (size_t)h * a.G + g;
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    __nv_bfloat16 *dst = a.out + head * DV + lane * PER;
+    __nv_bfloat16 *dst = a.out + head * DV + slice * SLICE + lane * PER;
 #pragma unroll
     for (int i = 0; i < PER; i += 2)
         *reinterpret_cast<uint32_t *>(dst + i) = pack_bf16x2(o[i] * inv, o[i + 1] * inv);
-    if (a.lse && lane == 0) a.lse[head] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+    if (a.lse && lane == 0 && slice == 0)
+        a.lse[head] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
 }
 
 template <int D, int NT>
@@ -411,7 +444,8 @@ cudaError_t launch_decode_gqa(const DecodeArgs &a, const CUtensorMap &tmK, const
 }
 
 cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl) {
-    const int64_t items = (int64_t)a.B * a.Hkv * a.G;
+    const int nslice = a.Dv > MERGE_DIMS ? a.Dv / MERGE_DIMS : 1;
+    const int64_t items = (int64_t)a.B * a.Hkv * a.G * nslice;
     const dim3 grid((unsigned)((items + 7) / 8));
     switch (a.Dv) {
         case 64: return launch_k(k_merge<64>, grid, dim3(256), 0, s, pdl, a);

@@ -7,37 +7,42 @@
 //
 // Geometry: 1 KV head, up to 16 query heads, Dqk = 576, Dv = 512.  The 16 heads fill the
 // M dimension of mma.m16n8k16, so the contraction is a real dense tile:
-//   S[16 heads x 16 tokens] = Q[16 x 576] . K^T      (36 k-steps)
-//   O[16 heads x 512 dims] += P[16 x 16] . V[16 x 512] (64 n-tiles)
-// Work: the selected pages are cut into 16-token tiles; the rows' tiles form one flat
+//   S[16 heads x 32 tokens] = Q[16 x 576] . K^T       (36 k-steps x 4 n-tiles)
+//   O[16 heads x 512 dims] += P[16 x 32] . V[32 x 512] (2 k-steps x 64 n-tiles)
+// Work: the selected pages are cut into 32-token tiles; the rows' tiles form one flat
 // list cut into W contiguous chunks, one chunk per 4-warp block (as in the GQA kernel,
 // partials go to slot row + chunk and are merged with the log-sum-exp rule).  All four
-// warps work on every tile: warp w contracts dims [144w, 144w+144) of Q.K^T, the four
-// partial S tiles are summed through shared memory (fixed order, so every warp holds the
-// same S), each warp runs the same online softmax and then owns output dims
-// [128w, 128w+128) of P.V.  K tiles (16 x 576 bf16 = 9 TMA boxes of 64 columns, 128-byte
-// swizzle) stream through a MLA_STAGES-deep ring filled by one elected thread; a stage is
-// refilled once every warp has passed the next tile's barrier.
+// warps work on every tile: warp w contracts dims [144w, 144w+144) of Q.K^T for all 32
+// tokens (four independent accumulation chains, one per 8-token n-tile), the four
+// partial S tiles are summed through shared memory in a fixed order (so every warp holds
+// the same S), each warp runs the same online softmax (skipping the output rescale when
+// no row maximum moved) and then owns output dims [128w, 128w+128) of P.V.  K tiles
+// (32 x 576 bf16 = 9 TMA boxes of 64 columns x 32 rows, 128-byte swizzle) stream through
+// a MLA_STAGES-deep ring filled by one elected thread; a stage is refilled once every warp
+// has passed the next tile's barrier.
 #include "vx_internal.h"
 
 namespace vx {
 
 constexpr int MLA_THREADS = 128;
-constexpr int MLA_STAGES = 4;
+constexpr int MLA_STAGES = 2;
 constexpr int MLA_DQK = 576, MLA_DV = 512;
-constexpr int MLA_KB = MLA_DQK / 64;                  // 9 boxes per tile
-constexpr int MLA_BOX = DEC_TILE * 128;               // 2 KB
-constexpr int MLA_TILE = MLA_KB * MLA_BOX;            // 18 KB
-constexpr int MLA_KSTEPS_PER_WARP = MLA_DQK / 16 / 4; // 9
-constexpr int MLA_NT_PER_WARP = MLA_DV / 8 / 4;       // 16 n-tiles of 8 dims
+constexpr int MLA_KB = MLA_DQK / 64;                   // 9 boxes per tile
+constexpr int MLA_BOX = MLA_TILE_TOKENS * 128;         // 4 KB (32 rows x 128 bytes)
+constexpr int MLA_TILE = MLA_KB * MLA_BOX;             // 36 KB
+constexpr int MLA_QBOX = 16 * 128;                     // Q: 16 head rows x 128 bytes
+constexpr int MLA_QBYTES = MLA_KB * MLA_QBOX;          // 18 KB
+constexpr int MLA_KSTEPS_PER_WARP = MLA_DQK / 16 / 4;  // 9
+constexpr int MLA_SNT = MLA_TILE_TOKENS / 8;           // 4 n-tiles of tokens in S
+constexpr int MLA_NT_PER_WARP = MLA_DV / 8 / 4;        // 16 n-tiles of output dims per warp
 
 struct MlaMeta {
-    int32_t row;     // -1: end of the chunk
+    int32_t row;  // -1: end of the chunk
     int32_t nvalid;
 };
 
 struct MlaShared {
-    float s_part[2][4][32][8];  // partial S per warp, per lane fragment (double buffered)
+    float4 s_part[2][4][MLA_SNT][32];  // partial S per warp and n-tile, per lane (double buffered)
     MlaMeta meta[MLA_STAGES];
     unsigned long long full[MLA_STAGES];
 };
@@ -60,8 +65,8 @@ __device__ __forceinline__ Resolved resolve_mla(const DecodeArgs &a, int64_t u, 
         set_err(a.err, VX_DATA_BAD_SELECTION);
         return rs;
     }
-    const int tok0 = j * a.P + sub * DEC_TILE;
-    const int nvalid = min(DEC_TILE, L - tok0);
+    const int tok0 = j * a.P + sub * MLA_TILE_TOKENS;
+    const int nvalid = min(MLA_TILE_TOKENS, L - tok0);
     if (nvalid <= 0) return rs;
     const int32_t phys = a.page_indices[a.page_ptr[b] + j];
     if (phys < 0 || phys >= a.num_pool_pages) {
@@ -69,10 +74,15 @@ __device__ __forceinline__ Resolved resolve_mla(const DecodeArgs &a, int64_t u, 
         return rs;
     }
     rs.z = phys;
-    rs.y = sub * DEC_TILE;
+    rs.y = sub * MLA_TILE_TOKENS;
     rs.nvalid = nvalid;
     rs.valid = true;
     return rs;
+}
+
+// keep-mask of a packed bf16 pair holding tokens t and t + 1
+__device__ __forceinline__ uint32_t pair_mask(int t, int nvalid) {
+    return (t < nvalid ? 0x0000ffffu : 0u) | (t + 1 < nvalid ? 0xffff0000u : 0u);
 }
 
 __global__ void __launch_bounds__(MLA_THREADS, 2)
@@ -80,9 +90,9 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const uint32_t sQ = base;                                   // 16 heads x 576, swizzled
-    const uint32_t sK0 = base + MLA_TILE;                       // MLA_STAGES tiles
-    MlaShared &sh = *reinterpret_cast<MlaShared *>(smem_raw + (base - raw) + (1 + MLA_STAGES) * MLA_TILE);
+    const uint32_t sK0 = base;                           // MLA_STAGES tiles
+    const uint32_t sQ = base + MLA_STAGES * MLA_TILE;    // 16 heads x 576, swizzled
+    MlaShared &sh = *reinterpret_cast<MlaShared *>(smem_raw + (base - raw) + MLA_STAGES * MLA_TILE + MLA_QBYTES);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g4 = lane >> 2, q4 = lane & 3;
     const int mi = lane >> 3, rr = lane & 7;
@@ -168,10 +178,12 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
 #pragma unroll
         for (int nt = 0; nt < MLA_NT_PER_WARP; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 4; e += 2) {
                 const int head = g4 + 8 * (e >> 1);
-                const int dim = warp * 128 + nt * 8 + 2 * q4 + (e & 1);
-                if (head < a.G) a.o_part[(slot * a.G + head) * MLA_DV + dim] = acc[nt][e];
+                const int dim = warp * 128 + nt * 8 + 2 * q4;
+                if (head < a.G)
+                    *reinterpret_cast<float2 *>(a.o_part + (slot * a.G + head) * MLA_DV + dim) =
+                        make_float2(acc[nt][e], acc[nt][e + 1]);
             }
         float lt[2];
 #pragma unroll
@@ -201,7 +213,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
             const int head = i / (MLA_DQK / 8), ch = i % (MLA_DQK / 8);
             uint4 v = make_uint4(0, 0, 0, 0);
             if (head < a.G) v = *reinterpret_cast<const uint4 *>(qb + (size_t)head * MLA_DQK + ch * 8);
-            const uint32_t dst = sQ + (ch >> 3) * MLA_BOX + swz128(head, ch & 7);
+            const uint32_t dst = sQ + (ch >> 3) * MLA_QBOX + swz128(head, ch & 7);
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
                          "r"(v.w)
                          : "memory");
@@ -239,35 +251,52 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
         const uint32_t sK = sK0 + (uint32_t)st * MLA_TILE;
         const int buf = it & 1;
 
-        // partial S over this warp's 144 dims
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // partial S over this warp's 144 dims, four 8-token n-tiles
+        float s[MLA_SNT][4];
+#pragma unroll
+        for (int nt = 0; nt < MLA_SNT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < MLA_KSTEPS_PER_WARP; ++kk) {
             const int kg = warp * MLA_KSTEPS_PER_WARP + kk;  // global 16-dim step
             const int box = kg >> 2, c0 = (kg & 3) * 2;
-            uint32_t qa0, qa1, qa2, qa3, kb0, kb1, kb2, kb3;
-            ldsm_x4(sQ + box * MLA_BOX + swz128(rr + 8 * (mi & 1), c0 + (mi >> 1)), qa0, qa1, qa2, qa3);
-            ldsm_x4(sK + box * MLA_BOX + swz128(rr + 8 * (mi >> 1), c0 + (mi & 1)), kb0, kb1, kb2, kb3);
-            mma_bf16_16816(s[0], qa0, qa1, qa2, qa3, kb0, kb1);
-            mma_bf16_16816(s[1], qa0, qa1, qa2, qa3, kb2, kb3);
+            uint32_t qa0, qa1, qa2, qa3;
+            ldsm_x4(sQ + box * MLA_QBOX + swz128(rr + 8 * (mi & 1), c0 + (mi >> 1)), qa0, qa1, qa2, qa3);
+#pragma unroll
+            for (int np = 0; np < MLA_SNT / 2; ++np) {  // pairs of token n-tiles
+                uint32_t kb0, kb1, kb2, kb3;
+                ldsm_x4(sK + box * MLA_BOX + swz128(np * 16 + rr + 8 * (mi >> 1), c0 + (mi & 1)), kb0, kb1, kb2, kb3);
+                mma_bf16_16816(s[2 * np], qa0, qa1, qa2, qa3, kb0, kb1);
+                mma_bf16_16816(s[2 * np + 1], qa0, qa1, qa2, qa3, kb2, kb3);
+            }
         }
-        float *mine = sh.s_part[buf][warp][lane];
-        reinterpret_cast<float4 *>(mine)[0] = make_float4(s[0][0], s[0][1], s[0][2], s[0][3]);
-        reinterpret_cast<float4 *>(mine)[1] = make_float4(s[1][0], s[1][1], s[1][2], s[1][3]);
+#pragma unroll
+        for (int nt = 0; nt < MLA_SNT; ++nt)
+            sh.s_part[buf][warp][nt][lane] = make_float4(s[nt][0], s[nt][1], s[nt][2], s[nt][3]);
         __syncthreads();
         // the stage used by the previous tile is free now: refill it
         if (warp == 0 && it > 0) issue(static_cast<int>((it - 1) % MLA_STAGES));
-        float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float x[MLA_SNT][4];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const float4 p0 = reinterpret_cast<const float4 *>(sh.s_part[buf][w][lane])[0];
-            const float4 p1 = reinterpret_cast<const float4 *>(sh.s_part[buf][w][lane])[1];
-            x[0][0] += p0.x; x[0][1] += p0.y; x[0][2] += p0.z; x[0][3] += p0.w;
-            x[1][0] += p1.x; x[1][1] += p1.y; x[1][2] += p1.z; x[1][3] += p1.w;
+        for (int nt = 0; nt < MLA_SNT; ++nt) {
+            float4 t = sh.s_part[buf][0][nt][lane];
+#pragma unroll
+            for (int w = 1; w < 4; ++w) {
+                const float4 p = sh.s_part[buf][w][nt][lane];
+                t.x += p.x;
+                t.y += p.y;
+                t.z += p.z;
+                t.w += p.w;
+            }
+            x[nt][0] = t.x;
+            x[nt][1] = t.y;
+            x[nt][2] = t.z;
+            x[nt][3] = t.w;
         }
-        // online softmax over the 16 tokens (columns), rows = heads g4 and g4 + 8
+        // online softmax over the 32 tokens (columns); rows = heads g4 and g4 + 8
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < MLA_SNT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int tok = nt * 8 + 2 * q4 + (e & 1);
@@ -276,48 +305,58 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
         float alpha[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-            float mx = fmaxf(fmaxf(x[0][2 * i], x[0][2 * i + 1]), fmaxf(x[1][2 * i], x[1][2 * i + 1]));
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < MLA_SNT; ++nt) mx = fmaxf(mx, fmaxf(x[nt][2 * i], x[nt][2 * i + 1]));
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
             const float m_new = fmaxf(m_run[i], mx);
             alpha[i] = exp2f(m_run[i] - m_new);
             m_run[i] = m_new;
         }
-        float p[2][4];
+        float p[MLA_SNT][4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < MLA_SNT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) p[nt][e] = exp2f(x[nt][e] - m_run[e >> 1]);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) l_run[i] = l_run[i] * alpha[i] + p[0][2 * i] + p[0][2 * i + 1] + p[1][2 * i] + p[1][2 * i + 1];
+        for (int i = 0; i < 2; ++i) {
+            float add = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < MLA_NT_PER_WARP; ++nt)
+            for (int nt = 0; nt < MLA_SNT; ++nt) add += p[nt][2 * i] + p[nt][2 * i + 1];
+            l_run[i] = l_run[i] * alpha[i] + add;
+        }
+        if (__any_sync(FULL, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] *= alpha[e >> 1];
-        // P as the A operand (rows = heads, k = tokens)
-        const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
-        const uint32_t pa1 = pack_bf16x2(p[0][2], p[0][3]);
-        const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
-        const uint32_t pa3 = pack_bf16x2(p[1][2], p[1][3]);
-        // O[:, warp dims] += P . V, V = first 512 dims of the K rows
-        const bool tail = nvalid < DEC_TILE;
-        const int t_lo = 2 * q4, t_hi = 8 + 2 * q4;
-        const uint32_t mlo = (t_lo < nvalid ? 0x0000ffffu : 0u) | (t_lo + 1 < nvalid ? 0xffff0000u : 0u);
-        const uint32_t mhi = (t_hi < nvalid ? 0x0000ffffu : 0u) | (t_hi + 1 < nvalid ? 0xffff0000u : 0u);
+            for (int nt = 0; nt < MLA_NT_PER_WARP; ++nt)
 #pragma unroll
-        for (int pr = 0; pr < MLA_NT_PER_WARP / 2; ++pr) {
-            const int ch = warp * 16 + pr * 2;  // 16-byte dim chunk of the first n-tile
-            const int box = ch >> 3, cc = ch & 7;
-            uint32_t v0, v1, v2, v3;
-            ldsm_x4_t(sK + box * MLA_BOX + swz128(rr + 8 * (mi & 1), cc + (mi >> 1)), v0, v1, v2, v3);
-            if (tail) {
-                v0 &= mlo;
-                v1 &= mhi;
-                v2 &= mlo;
-                v3 &= mhi;
+                for (int e = 0; e < 4; ++e) acc[nt][e] *= alpha[e >> 1];
+        }
+        // O[:, warp dims] += P . V over two 16-token k-steps; V = first 512 dims of the K rows
+        const bool tail = nvalid < MLA_TILE_TOKENS;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const uint32_t pa0 = pack_bf16x2(p[2 * ks][0], p[2 * ks][1]);
+            const uint32_t pa1 = pack_bf16x2(p[2 * ks][2], p[2 * ks][3]);
+            const uint32_t pa2 = pack_bf16x2(p[2 * ks + 1][0], p[2 * ks + 1][1]);
+            const uint32_t pa3 = pack_bf16x2(p[2 * ks + 1][2], p[2 * ks + 1][3]);
+            const uint32_t mlo = pair_mask(ks * 16 + 2 * q4, nvalid);
+            const uint32_t mhi = pair_mask(ks * 16 + 8 + 2 * q4, nvalid);
+#pragma unroll
+            for (int pr = 0; pr < MLA_NT_PER_WARP / 2; ++pr) {
+                const int ch = warp * 16 + pr * 2;  // 16-byte dim chunk of the first n-tile
+                const int box = ch >> 3, cc = ch & 7;
+                uint32_t v0, v1, v2, v3;
+                ldsm_x4_t(sK + box * MLA_BOX + swz128(ks * 16 + rr + 8 * (mi & 1), cc + (mi >> 1)), v0, v1, v2, v3);
+                if (tail) {
+                    v0 &= mlo;
+                    v1 &= mhi;
+                    v2 &= mlo;
+                    v3 &= mhi;
+                }
+                mma_bf16_16816(acc[2 * pr], pa0, pa1, pa2, pa3, v0, v1);
+                mma_bf16_16816(acc[2 * pr + 1], pa0, pa1, pa2, pa3, v2, v3);
             }
-            mma_bf16_16816(acc[2 * pr], pa0, pa1, pa2, pa3, v0, v1);
-            mma_bf16_16816(acc[2 * pr + 1], pa0, pa1, pa2, pa3, v2, v3);
         }
     }
 
@@ -336,7 +375,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
 }
 
 cudaError_t launch_decode_mla(const DecodeArgs &a, const CUtensorMap &tmK, int grid, cudaStream_t s, bool pdl) {
-    const size_t smem = 1024 + (size_t)(1 + MLA_STAGES) * MLA_TILE + sizeof(MlaShared);
+    const size_t smem = 1024 + (size_t)MLA_STAGES * MLA_TILE + MLA_QBYTES + sizeof(MlaShared);
     static std::atomic<unsigned long long> done;
     cudaError_t e = ensure_smem_limit(k_decode_mla, (int)smem, done);
     if (e != cudaSuccess) return e;

@@ -4,120 +4,320 @@
 // current query with the cached centroids; the MLA experiment section scores on the
 // 576-dim latent + rope key (rope-aware) and, as a variant, on the 512 latent dims.
 //
-// The contraction over the G query heads of a KV group is done first (fp32, exact for a
-// few bf16 values), so the kernel is a GEMV per (request, KV head): it streams each
-// page's centroid row (all KV heads contiguous, Hkv * Dqk bf16) once with 16-byte
-// non-coherent loads, several pages in flight per warp.  Each lane keeps the summed
-// query for the 8 dims it multiplies in registers; partial dots of one head are
-// combined with XOR shuffles inside the lane segment that covers that head.
+// The contraction over the G query heads of a KV group is done first (fp32), so the
+// kernel is a GEMV per (request, KV head) that must stream every page's centroid row
+// (all KV heads contiguous, Hkv * Dqk bf16) exactly once at HBM speed.
+//
+// Work layout: a persistent grid of one block of SCORE_WARPS warps per SM; all pages of
+// all requests form one flat list (each block derives the per-request page prefix from
+// seq_lens), and every warp takes an equal contiguous range of it.
+// Data path: each warp owns a ring of SCORE_STAGES stages in shared memory; a stage
+// holds up to PPS consecutive pages of one request, each page row fetched by one 1-D TMA
+// bulk copy (completion counted on the stage's mbarrier).
+// Compute: lane l works on page l / (Hkv*S) of the stage, KV head (l / S) % Hkv and
+// segment l % S of that head's row (DPL = D / S dims, kept as the summed query in
+// registers), so a dot product is DPL FMAs plus a log2(S)-step shuffle; each lane walks
+// its 16-byte chunks in an order rotated by its lane id, which keeps the shared-memory
+// reads free of bank conflicts.  Scores are collected in a per-warp [Hkv][32] buffer and
+// written as coalesced 128-byte rows.
 #include "vx_internal.h"
 
 namespace vx {
 
-constexpr int SCORE_MAX_ITS = 4;  // 16-byte loads per lane per page (Hkv * Dqk <= 1024)
+constexpr int SCORE_STAGES = 4;        // stages in flight per warp
+constexpr int SCORE_MAX_BATCH = 4096;  // requests whose prefix fits the block's shared memory
+constexpr int SCORE_MAX_HKV = 16;
 
+// dims per lane for a head dim (the head row is split over D / DPL lanes)
 template <int D>
-__global__ void __launch_bounds__(SCORE_WARPS * 32) k_score_pages(ScoreArgs a) {
-    pdl_launch_dependents();
-    pdl_wait();  // q and the centroids may be written by the previous kernel
-    constexpr int CH = D / 8;                 // 16-byte chunks per head row
-    constexpr bool SEGMENTED = CH <= 32;      // a head row fits in a lane segment
-    const int b = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t L = a.seq_lens[b];
-    if (L < 1 || L > a.max_pages * a.P) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
-        return;
-    }
-    const int n = ceil_div(L, a.P);
-    const int j_lo = blockIdx.x * SCORE_PAGES_PER_BLOCK;
-    if (j_lo >= n) return;
-    const int j_hi = min(n, j_lo + SCORE_PAGES_PER_BLOCK);
-    const int E = a.Hkv * CH;  // chunks per page row
+struct ScoreSplit {
+    static constexpr int DPL = D == 576 ? 72 : (D == 128 ? 64 : 32);
+    static constexpr int S = D / DPL;    // lanes per head row
+    static constexpr int NCH = DPL / 8;  // 16-byte chunks per lane
+};
 
-    extern __shared__ float qsum[];  // [Hkv][D]
-    for (int i = threadIdx.x; i < a.Hkv * D; i += blockDim.x) {
-        const int h = i / D, d = i % D;
-        float s = 0.f;
-        if (d < a.score_dims) {
-            const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)h * a.G) * D + d;
-            for (int g = 0; g < a.G; ++g) s += __bfloat162float(qb[(size_t)g * D]);
-        }
-        qsum[i] = s;
+struct ScoreMeta {
+    int32_t b, j, n;  // request, first logical page, pages in the stage
+};
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Block-wide exclusive scan over SCORE_WARPS warps; `tmp` holds SCORE_WARPS ints.
+__device__ __forceinline__ int score_block_scan(int v, int *tmp, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(FULL, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) tmp[warp] = x;
+    __syncthreads();
+    int before = 0;
+    total = 0;
+#pragma unroll
+    for (int w = 0; w < SCORE_WARPS; ++w) {
+        const int t = tmp[w];
+        if (w < warp) before += t;
+        total += t;
     }
     __syncthreads();
+    return before + x - v;
+}
 
-    // this lane's chunks are the same for every page: keep their query values in registers
-    float qreg[SCORE_MAX_ITS][8];
-#pragma unroll
-    for (int it = 0; it < SCORE_MAX_ITS; ++it) {
-        const int ci = it * 32 + lane;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qreg[it][i] = (ci < E) ? qsum[ci * 8 + i] : 0.f;
+template <int D>
+__global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a) {
+    pdl_launch_dependents();
+    pdl_wait();  // q, the table and the centroids may come from the previous kernel
+    using SP = ScoreSplit<D>;
+    constexpr int DPL = SP::DPL, S = SP::S, NCH = SP::NCH;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lanes_per_page = a.Hkv * S;        // divides 32 (checked on the host)
+    const int pps = 32 / lanes_per_page;         // pages per stage
+    const uint32_t row_bytes = (uint32_t)a.Hkv * D * 2u;
+    const uint32_t stage_bytes = ((uint32_t)pps * row_bytes + 127u) & ~127u;
+    const int my_page = lane / lanes_per_page;
+    const int my_head = (lane / S) % a.Hkv;
+    const int my_seg = lane % S;
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    int *prefix = reinterpret_cast<int *>(smem);  // B + 1: pages of request b = [prefix[b], prefix[b+1])
+    int *pptr = prefix + a.B + 1;                 // B: page_ptr
+    const uint32_t head_bytes = ((uint32_t)(2 * a.B + 1) * 4u + 127u) & ~127u;
+    uint8_t *per_warp = smem + head_bytes + (size_t)warp * (SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 +
+                                                            SCORE_STAGES * (8 + sizeof(ScoreMeta)));
+    const uint32_t ring0 = smem_u32(per_warp);
+    float *tbuf = reinterpret_cast<float *>(per_warp + SCORE_STAGES * stage_bytes);  // [Hkv][32]
+    const uint32_t bar0 = smem_u32(per_warp + SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4);
+    ScoreMeta *meta = reinterpret_cast<ScoreMeta *>(per_warp + SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 +
+                                                    SCORE_STAGES * 8);
+    __shared__ int scan_tmp[SCORE_WARPS];
+
+    if (lane == 0) {
+        for (int s = 0; s < SCORE_STAGES; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
     }
+    {   // per-request page prefix and row starts
+        const int per = ceil_div(a.B, blockDim.x);
+        const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
+        int local = 0;
+        for (int b = b0; b < b1; ++b) {
+            const int32_t L = a.seq_lens[b];
+            const bool ok = L >= 1 && L <= a.max_pages * a.P;
+            if (!ok && blockIdx.x == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
+            local += ok ? ceil_div(L, a.P) : 0;
+            pptr[b] = a.page_ptr[b];
+        }
+        int total;
+        int run = score_block_scan(local, scan_tmp, total);
+        for (int b = b0; b < b1; ++b) {
+            prefix[b] = run;
+            const int32_t L = a.seq_lens[b];
+            run += (L >= 1 && L <= a.max_pages * a.P) ? ceil_div(L, a.P) : 0;
+        }
+        if (threadIdx.x == 0) prefix[a.B] = total;
+        __syncthreads();
+    }
+    const int64_t T = prefix[a.B];
+    const int64_t W = (int64_t)gridDim.x * SCORE_WARPS;
+    const int64_t wid = (int64_t)blockIdx.x * SCORE_WARPS + warp;
+    const int64_t p_begin = wid * T / W, p_end = (wid + 1) * T / W;
+    if (p_begin >= p_end) return;
 
-    const int32_t *row = a.page_indices + a.page_ptr[b];
-    for (int jb = j_lo + warp * SCORE_UNROLL; jb < j_hi; jb += SCORE_WARPS * SCORE_UNROLL) {
-        int32_t phys[SCORE_UNROLL];
-        uint4 v[SCORE_UNROLL][SCORE_MAX_ITS];
-#pragma unroll
-        for (int u = 0; u < SCORE_UNROLL; ++u) {
-            const int j = jb + u;
-            phys[u] = -1;
-            if (j < j_hi) {
-                const int32_t p = row[j];
-                if (p >= 0 && p < a.num_pool_pages) phys[u] = p;
-                else if (lane == 0) set_err(a.err, VX_DATA_BAD_PAGE_ID);
-            }
+    // lane resolves flat page p: request, logical page, physical page (-1: skip)
+    auto resolve = [&](int64_t p, int32_t &rb, int32_t &rj) -> int32_t {
+        rb = -1;
+        rj = 0;
+        if (p >= p_end) return -1;
+        int lo = 0, hi = a.B - 1;  // last b with prefix[b] <= p
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= p) lo = mid;
+            else hi = mid - 1;
         }
-#pragma unroll
-        for (int u = 0; u < SCORE_UNROLL; ++u) {
-            const __nv_bfloat16 *c = a.centroids + (size_t)max(phys[u], 0) * a.Hkv * D;
-#pragma unroll
-            for (int it = 0; it < SCORE_MAX_ITS; ++it) {
-                const int ci = it * 32 + lane;
-                v[u][it] = (phys[u] >= 0 && ci < E) ? ld_nc_v4(c + ci * 8) : make_uint4(0, 0, 0, 0);
-            }
+        rb = lo;
+        rj = static_cast<int32_t>(p - prefix[lo]);
+        const int32_t id = a.page_indices[pptr[lo] + rj];
+        if (id < 0 || id >= a.num_pool_pages) {
+            set_err(a.err, VX_DATA_BAD_PAGE_ID);
+            return -1;
         }
+        return id;
+    };
+
+    // summed query of request b for this lane's head and segment, in the lane's chunk order
+    float qreg[NCH][8];
+    auto load_query = [&](int b) {
+        const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)my_head * a.G) * D + my_seg * DPL;
 #pragma unroll
-        for (int u = 0; u < SCORE_UNROLL; ++u) {
-            if (phys[u] < 0) continue;  // warp-uniform
-            const int j = jb + u;
-            float tot = 0.f;
+        for (int c = 0; c < NCH; ++c) {
+            const int ch = (c + lane) % NCH;  // rotated chunk order
 #pragma unroll
-            for (int it = 0; it < SCORE_MAX_ITS; ++it) {
-                if (it * 32 >= E) break;
-                float f[8];
-                bf16x8_to_f32(v[u][it], f);
-                float dot = 0.f;
+            for (int i = 0; i < 8; ++i) qreg[c][i] = 0.f;
+            if (my_seg * DPL + ch * 8 < a.score_dims) {
+                for (int g = 0; g < a.G; ++g) {
+                    float f[8];
+                    bf16x8_to_f32(ld_nc_v4(qb + (size_t)g * D + ch * 8), f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) dot = fmaf(f[i], qreg[it][i], dot);
-                if constexpr (SEGMENTED) {
-#pragma unroll
-                    for (int off = CH / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(FULL, dot, off);
-                    const int ci = it * 32 + lane;
-                    if ((lane % CH) == 0 && ci < E) {
-                        const int h = ci / CH;
-                        a.scores[((size_t)b * a.Hkv + h) * a.max_pages + j] = dot;
-                    }
-                } else {
-                    tot += dot;
+                    for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
                 }
             }
-            if constexpr (!SEGMENTED) {
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(FULL, tot, off);
-                if (lane == 0) a.scores[(size_t)b * a.Hkv * a.max_pages + j] = tot;  // Hkv == 1
+        }
+    };
+
+    // score transpose buffer: window of 32 logical pages [wj, wj + 32) of request wb
+    int wb = -1, wj = 0;
+    uint32_t wmask = 0;
+    auto flush_window = [&]() {
+        __syncwarp();
+        if (wmask) {
+            float *dst = a.scores + (size_t)wb * a.Hkv * a.max_pages + wj + lane;
+            const bool mine = (wmask >> lane) & 1u;
+            for (int h = 0; h < a.Hkv; ++h)
+                if (mine) dst[(size_t)h * a.max_pages] = tbuf[h * 32 + lane];
+        }
+        __syncwarp();
+        wmask = 0;
+    };
+
+    int64_t batch = p_begin;
+    int32_t my_b, my_j;
+    int32_t my_id = resolve(batch + lane, my_b, my_j);
+    uint32_t pending = __ballot_sync(FULL, my_id >= 0);
+    uint32_t issued = 0, consumed = 0;
+    bool failed = false;
+    int cur_b = -1;
+    for (;;) {
+        // fill stages: up to pps consecutive pending pages of one request each
+        while (issued - consumed < SCORE_STAGES) {
+            if (pending == 0) {
+                batch += 32;
+                if (batch >= p_end) break;
+                my_id = resolve(batch + lane, my_b, my_j);
+                pending = __ballot_sync(FULL, my_id >= 0);
+                continue;
             }
+            const int st = static_cast<int>(issued % SCORE_STAGES);
+            const uint32_t bar = bar0 + 8u * st;
+            const uint32_t dst = ring0 + (uint32_t)st * stage_bytes;
+            // choose the stage's pages (warp-uniform): lanes of `pending`, in order
+            uint32_t take = 0;
+            int n = 0, sb = -1, sj = 0;
+            while (n < pps && pending) {
+                const int src = __ffs(pending) - 1;
+                const int32_t rb = __shfl_sync(FULL, my_b, src);
+                const int32_t rj = __shfl_sync(FULL, my_j, src);
+                if (n > 0 && (rb != sb || rj != sj + n)) break;  // one request, consecutive pages
+                if (n == 0) {
+                    sb = rb;
+                    sj = rj;
+                }
+                take |= 1u << src;
+                pending &= pending - 1;
+                ++n;
+            }
+            if (lane == 0) {
+                meta[st].b = sb;
+                meta[st].j = sj;
+                meta[st].n = n;
+                mbar_arrive_expect_tx(bar, (uint32_t)n * row_bytes);  // all bytes announced first
+            }
+            __syncwarp();
+            if ((take >> lane) & 1u) {
+                const uint32_t slot = __popc(take & ((1u << lane) - 1u));
+                fence_proxy_async_smem();  // earlier generic reads of this stage come first
+                bulk_load(dst + slot * row_bytes, a.centroids + (size_t)my_id * a.Hkv * D, row_bytes, bar);
+            }
+            __syncwarp();
+            ++issued;
+        }
+        if (consumed == issued) break;
+        const int st = static_cast<int>(consumed % SCORE_STAGES);
+        const bool ok = __all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / SCORE_STAGES) & 1u));
+        if (!ok) {
+            failed = true;
+            break;
+        }
+        const ScoreMeta m = meta[st];
+        if (m.b != cur_b) {
+            load_query(m.b);
+            cur_b = m.b;
+        }
+        // dot products: this lane's (page, head, segment)
+        float dot = 0.f;
+        if (my_page < m.n) {
+            const uint32_t src = ring0 + (uint32_t)st * stage_bytes + (uint32_t)my_page * row_bytes +
+                                 (uint32_t)(my_head * D + my_seg * DPL) * 2u;
+            float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                const int ch = (c + lane) % NCH;
+                uint4 v;
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                             : "r"(src + (uint32_t)ch * 16u));
+                float f[8];
+                bf16x8_to_f32(v, f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc4[i & 3] = fmaf(f[i], qreg[c][i], acc4[i & 3]);
+            }
+            dot = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+        }
+#pragma unroll
+        for (int off = 1; off < S; off <<= 1) dot += __shfl_xor_sync(FULL, dot, off);
+        __syncwarp();  // every lane is done with this stage before it is refilled
+        ++consumed;
+        // record the stage's scores in the transpose window (a stage spans at most two
+        // 32-page windows since pps <= 16)
+        const int jpage = m.j + my_page;
+        for (int part = 0; part < 2; ++part) {
+            const int lo = part == 0 ? m.j : ((m.j & ~31) + 32);
+            const int hi = min(m.j + m.n, (lo & ~31) + 32);
+            if (lo >= hi) break;
+            if (m.b != wb || (lo & ~31) != wj) {
+                flush_window();
+                wb = m.b;
+                wj = lo & ~31;
+            }
+            if (my_seg == 0 && my_page < m.n && jpage >= lo && jpage < hi) tbuf[my_head * 32 + (jpage - wj)] = dot;
+            const int cnt = hi - lo;
+            wmask |= (cnt >= 32 ? 0xffffffffu : ((1u << cnt) - 1u)) << (lo - wj);
         }
     }
+    if (failed) {
+        if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
+        for (uint32_t i = consumed; i < issued; ++i)
+            (void)mbar_wait_bounded(bar0 + 8u * (i % SCORE_STAGES), (i / SCORE_STAGES) & 1u);
+        return;
+    }
+    flush_window();
 }
 
 template <int D>
 static cudaError_t launch_score_d(const ScoreArgs &a, cudaStream_t s, bool pdl) {
-    dim3 grid((a.max_pages + SCORE_PAGES_PER_BLOCK - 1) / SCORE_PAGES_PER_BLOCK, a.B);
-    const size_t smem = sizeof(float) * a.Hkv * D;
-    return launch_k(k_score_pages<D>, grid, dim3(SCORE_WARPS * 32), smem, s, pdl, a);
+    using SP = ScoreSplit<D>;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int lpp = a.Hkv * SP::S;
+    if (a.B > SCORE_MAX_BATCH || a.Hkv > SCORE_MAX_HKV || lpp > 32 || 32 % lpp) return cudaErrorInvalidValue;
+    const size_t row_bytes = (size_t)a.Hkv * D * 2;
+    const size_t stage_bytes = ((32 / lpp) * row_bytes + 127) & ~size_t(127);
+    const size_t head = ((size_t)(2 * a.B + 1) * 4 + 127) & ~size_t(127);
+    const size_t per_warp = SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 + SCORE_STAGES * (8 + sizeof(ScoreMeta));
+    const size_t smem = head + (size_t)SCORE_WARPS * per_warp;
+    // largest need: 4096 requests' prefix (32.9 KB) + 8 warps x 20.6 KB (MLA stages) < 200 KB
+    constexpr int SCORE_SMEM_LIMIT = 200 * 1024;
+    if (smem > (size_t)SCORE_SMEM_LIMIT) return cudaErrorInvalidValue;
+    static std::atomic<unsigned long long> done;
+    e = ensure_smem_limit(k_score_pages<D>, SCORE_SMEM_LIMIT, done);
+    if (e != cudaSuccess) return e;
+    return launch_k(k_score_pages<D>, dim3(sms), dim3(SCORE_WARPS * 32), smem, s, pdl, a);
 }
 
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s, bool pdl) {

@@ -4,11 +4,12 @@
 // stage, with stochastic early termination and remapping as the faster approximate
 // form (its kernel-ablation section reports recall@k > 0.97 for that form).
 //
-// One 1024-thread block per row.  Scores become order-preserving uint32 keys (-0.0
-// folded onto +0.0), kept in shared memory when the row fits.
-//   exact:  MSB-first radix select, 8-bit digits, 256-bin shared histograms; the digit
-//           holding the k-th largest key is found with a warp suffix scan; the search
-//           stops early once the boundary bucket holds exactly the slots left.
+// One block per row (256 threads for rows up to TOPK_SMALL_MAX pages, 1024 beyond).
+// Scores become order-preserving uint32 keys (-0.0 folded onto +0.0), kept in shared
+// memory when the row fits.
+//   exact:  MSB-first radix select with 11/11/10-bit digits: a shared histogram per
+//           digit, the digit holding the k-th largest key found by a block suffix scan,
+//           early exit once the boundary bucket holds exactly the slots left.
 //   approx: fp32 remap of each score to a 12-bit code between the row's min and max,
 //           one 4096-bin histogram, the boundary code b* from a block suffix scan, no
 //           refinement: the slots left are filled from code b* in cyclic page order from
@@ -20,6 +21,9 @@
 #include "vx_internal.h"
 
 namespace vx {
+
+constexpr int TOPK_SMALL_MAX = 4096;  // rows up to this many pages use 256-thread blocks
+constexpr int TOPK_HIST = 1 << APPROX_BITS;
 
 __device__ __forceinline__ uint32_t order_key(float s) {
     uint32_t f = __float_as_uint(s);
@@ -35,9 +39,11 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t i) {
     return z ^ (z >> 31);
 }
 
-// Block-wide exclusive scan of one int per thread (TOPK_THREADS threads); also returns
-// the total.  `tmp` holds 32 ints of shared memory.  Contains __syncthreads.
+// Block-wide exclusive scan of one int per thread; also returns the total.  `tmp` holds
+// 32 ints of shared memory.  Contains __syncthreads.
+template <int THREADS>
 __device__ __forceinline__ int block_exclusive_scan(int v, int *tmp, int &total) {
+    constexpr int NW = THREADS / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
 #pragma unroll
@@ -48,30 +54,52 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *tmp, int &total)
     if (lane == 31) tmp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = tmp[lane];
+        int w = lane < NW ? tmp[lane] : 0;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int y = __shfl_up_sync(FULL, w, off);
             if (lane >= off) w += y;
         }
-        tmp[lane] = w;  // inclusive over warps
+        if (lane < NW) tmp[lane] = w;  // inclusive over warps
     }
     __syncthreads();
-    total = tmp[31];
+    total = tmp[NW - 1];
     const int before = (warp > 0 ? tmp[warp - 1] : 0) + x - v;
     __syncthreads();  // tmp may be reused right after
     return before;
 }
 
 struct TopkShared {
-    int hist[1 << APPROX_BITS];
+    int hist[TOPK_HIST];
     int scan_tmp[32];
     int bcast[4];
     float fmin[32], fmax[32];
 };
 
-template <bool APPROX>
-__global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
+// The bin holding the `need`-th largest element of the first `bins` histogram entries,
+// searching from the top: writes (bin, count above it, its count) to sh.bcast.
+template <int THREADS>
+__device__ __forceinline__ void block_find_bin(TopkShared &sh, int bins, int need) {
+    const int per = bins / THREADS;  // bins per thread (bins is a multiple of THREADS)
+    const int base = (THREADS - 1 - (int)threadIdx.x) * per;  // thread 0 owns the top bins
+    int own = 0;
+    for (int i = 0; i < per; ++i) own += sh.hist[base + i];
+    int total;
+    int above = block_exclusive_scan<THREADS>(own, sh.scan_tmp, total);
+    for (int i = per - 1; i >= 0; --i) {
+        const int c = sh.hist[base + i];
+        if (above < need && above + c >= need) {
+            sh.bcast[0] = base + i;
+            sh.bcast[1] = above;
+            sh.bcast[2] = c;
+        }
+        above += c;
+    }
+    __syncthreads();
+}
+
+template <bool APPROX, int THREADS>
+__global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
     pdl_launch_dependents();
     pdl_wait();  // the scores are written by the previous kernel
     __shared__ TopkShared sh;
@@ -82,24 +110,23 @@ __global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
     const float *row = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages;
     const int32_t L = a.seq_lens[b];
     if (L < 1 || L > a.max_pages * a.P) {
-        for (int i = tid; i < a.k; i += TOPK_THREADS) out[i] = -1;
+        for (int i = tid; i < a.k; i += THREADS) out[i] = -1;
         if (tid == 0 && h == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
         return;
     }
     const int n = ceil_div(L, a.P);
     const int keff = min(a.k, n);
     if (keff == n) {  // every page is chosen
-        for (int i = tid; i < a.k; i += TOPK_THREADS) out[i] = i < n ? i : -1;
+        for (int i = tid; i < a.k; i += THREADS) out[i] = i < n ? i : -1;
         return;
     }
     const bool in_smem = n <= a.smem_keys;
 
     // per-thread contiguous run [r0, r1) used by the ordered compaction
-    const int per = ceil_div(n, TOPK_THREADS);
+    const int per = ceil_div(n, THREADS);
     const int r0 = min(n, tid * per), r1 = min(n, r0 + per);
 
-    // -------- key of page j: radix key (exact) or remap code (approx)
-    uint32_t prefix = 0, mask = 0;  // exact: chosen iff (key & mask) > prefix, or == and rank < remaining
+    uint32_t prefix = 0, mask = 0;  // chosen iff (key & mask) > prefix, or == and rank < remaining
     int remaining = keff;           // slots to take from the boundary bucket
     int offset = 0;                 // approx: start of the cyclic fill
     float lo = 0.f, scale = 0.f;
@@ -107,53 +134,32 @@ __global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
 
     if constexpr (!APPROX) {
         if (in_smem)
-            for (int j = tid; j < n; j += TOPK_THREADS) skeys[j] = order_key(row[j]);
+            for (int j = tid; j < n; j += THREADS) skeys[j] = order_key(row[j]);
         __syncthreads();
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += TOPK_THREADS) sh.hist[i] = 0;
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass) {
+            const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+            const int bins = pass == 2 ? 1024 : 2048;
+            const uint32_t dmask = (uint32_t)bins - 1u;
+            for (int i = tid; i < bins; i += THREADS) sh.hist[i] = 0;
             __syncthreads();
-            for (int j = tid; j < n; j += TOPK_THREADS) {
+            for (int j = tid; j < n; j += THREADS) {
                 const uint32_t key = in_smem ? skeys[j] : order_key(row[j]);
-                if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
+                if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & dmask], 1);
             }
             __syncthreads();
-            if (warp == 0) {
-                // lane owns digits [8*lane, 8*lane+8); suffix sums from the top digit down
-                int c[8], own = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    c[i] = sh.hist[lane * 8 + i];
-                    own += c[i];
-                }
-                int suf = own;  // inclusive suffix over lanes >= lane
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int y = __shfl_down_sync(FULL, suf, off);
-                    if (lane + off < 32) suf += y;
-                }
-                int above = suf - own;  // digits owned by higher lanes
-#pragma unroll
-                for (int i = 7; i >= 0; --i) {
-                    if (above < remaining && above + c[i] >= remaining) {
-                        sh.bcast[0] = lane * 8 + i;
-                        sh.bcast[1] = above;
-                        sh.bcast[2] = c[i];
-                    }
-                    above += c[i];
-                }
-            }
-            __syncthreads();
+            block_find_bin<THREADS>(sh, bins, remaining);
             const int digit = sh.bcast[0], above = sh.bcast[1], cnt = sh.bcast[2];
             remaining -= above;
             prefix |= static_cast<uint32_t>(digit) << shift;
-            mask |= 0xffu << shift;
+            mask |= dmask << shift;
             __syncthreads();
             if (cnt == remaining) break;  // the whole boundary bucket is taken
         }
     } else {
         // row min / max
         float mn = INFINITY, mx = -INFINITY;
-        for (int j = tid; j < n; j += TOPK_THREADS) {
+        for (int j = tid; j < n; j += THREADS) {
             const float s = row[j];
             mn = fminf(mn, s);
             mx = fmaxf(mx, s);
@@ -167,47 +173,29 @@ __global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
             sh.fmin[warp] = mn;
             sh.fmax[warp] = mx;
         }
-        for (int i = tid; i < (1 << APPROX_BITS); i += TOPK_THREADS) sh.hist[i] = 0;
+        for (int i = tid; i < TOPK_HIST; i += THREADS) sh.hist[i] = 0;
         __syncthreads();
         mn = sh.fmin[0];
         mx = sh.fmax[0];
-        for (int w = 1; w < TOPK_THREADS / 32; ++w) {
+        for (int w = 1; w < THREADS / 32; ++w) {
             mn = fminf(mn, sh.fmin[w]);
             mx = fmaxf(mx, sh.fmax[w]);
         }
         lo = mn;
         const float range = __fsub_rn(mx, mn);
-        scale = __fdiv_rn(static_cast<float>(1 << APPROX_BITS), range);
+        scale = __fdiv_rn(static_cast<float>(TOPK_HIST), range);
         flat = !(mx > mn) || isinf(scale);
-        for (int j = tid; j < n; j += TOPK_THREADS) {
+        for (int j = tid; j < n; j += THREADS) {
             uint32_t code = 0;
             if (!flat) {
-                const float t = __fmul_rn(__fsub_rn(row[j], lo), scale);
-                const float f = floorf(t);
-                code = f >= float((1 << APPROX_BITS) - 1) ? (1u << APPROX_BITS) - 1 : static_cast<uint32_t>(f);
+                const float f = floorf(__fmul_rn(__fsub_rn(row[j], lo), scale));
+                code = f >= float(TOPK_HIST - 1) ? TOPK_HIST - 1 : static_cast<uint32_t>(f);
             }
             if (in_smem) skeys[j] = code;
             atomicAdd(&sh.hist[code], 1);
         }
         __syncthreads();
-        // boundary code: suffix scan of 4096 bins, 4 per thread, highest bins first
-        constexpr int BPT = (1 << APPROX_BITS) / TOPK_THREADS;
-        const int base = (TOPK_THREADS - 1 - tid) * BPT;  // thread 0 owns the top bins
-        int own = 0;
-#pragma unroll
-        for (int i = 0; i < BPT; ++i) own += sh.hist[base + i];
-        int total;
-        int above = block_exclusive_scan(own, sh.scan_tmp, total);
-#pragma unroll
-        for (int i = BPT - 1; i >= 0; --i) {
-            const int c = sh.hist[base + i];
-            if (above < keff && above + c >= keff) {
-                sh.bcast[0] = base + i;
-                sh.bcast[1] = above;
-            }
-            above += c;
-        }
-        __syncthreads();
+        block_find_bin<THREADS>(sh, TOPK_HIST, keff);
         prefix = static_cast<uint32_t>(sh.bcast[0]);
         mask = 0xffffffffu;
         remaining = keff - sh.bcast[1];
@@ -219,7 +207,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
         if constexpr (APPROX) {
             if (flat) return 0u;
             const float f = floorf(__fmul_rn(__fsub_rn(row[j], lo), scale));
-            return f >= float((1 << APPROX_BITS) - 1) ? (1u << APPROX_BITS) - 1 : static_cast<uint32_t>(f);
+            return f >= float(TOPK_HIST - 1) ? TOPK_HIST - 1 : static_cast<uint32_t>(f);
         } else {
             return order_key(row[j]);
         }
@@ -235,11 +223,11 @@ __global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
         }
     }
     int eq_total;
-    const int eq_before = block_exclusive_scan(eq_local, sh.scan_tmp, eq_total);
+    const int eq_before = block_exclusive_scan<THREADS>(eq_local, sh.scan_tmp, eq_total);
     int eq_before_offset = 0;
     if constexpr (APPROX) {
         int tmp_total;
-        block_exclusive_scan(eq_before_offset_local, sh.scan_tmp, tmp_total);
+        block_exclusive_scan<THREADS>(eq_before_offset_local, sh.scan_tmp, tmp_total);
         eq_before_offset = tmp_total;  // members with page index < offset
     }
     // pass 2: chosen flags, counted per run
@@ -261,7 +249,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
         }
     }
     int sel_total;
-    int pos = block_exclusive_scan(sel_local, sh.scan_tmp, sel_total);
+    int pos = block_exclusive_scan<THREADS>(sel_local, sh.scan_tmp, sel_total);
     {
         int eq_rank = eq_before;
         for (int j = r0; j < r1; ++j) {
@@ -273,17 +261,23 @@ __global__ void __launch_bounds__(TOPK_THREADS) k_topk(TopkArgs a) {
             if ((key & mask) == prefix) ++eq_rank;
         }
     }
-    for (int i = sel_total + tid; i < a.k; i += TOPK_THREADS) out[i] = -1;
+    for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;
 }
 
-cudaError_t launch_topk(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
-    dim3 grid(a.Hkv, a.B);
+template <int THREADS>
+static cudaError_t launch_topk_t(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
+    const dim3 grid(a.Hkv, a.B);
     const size_t smem = sizeof(uint32_t) * (size_t)a.smem_keys;
-    auto kern = mode == 0 ? k_topk<false> : k_topk<true>;
+    auto kern = mode == 0 ? k_topk<false, THREADS> : k_topk<true, THREADS>;
     static std::atomic<unsigned long long> done[2];
     cudaError_t e = ensure_smem_limit(kern, (int)(sizeof(uint32_t) * TOPK_SMEM_KEYS), done[mode]);
     if (e != cudaSuccess) return e;
-    return launch_k(kern, grid, dim3(TOPK_THREADS), smem, s, pdl, a);
+    return launch_k(kern, grid, dim3(THREADS), smem, s, pdl, a);
+}
+
+cudaError_t launch_topk(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
+    if (a.max_pages <= TOPK_SMALL_MAX) return launch_topk_t<256>(a, mode, s, pdl);
+    return launch_topk_t<1024>(a, mode, s, pdl);
 }
 
 }  // namespace vx

@@ -55,18 +55,21 @@ vx_status check_geometry(const vx_geometry *g) {
     const int G = g->num_q_heads / g->num_kv_heads;
     if (g->page_size != 16 && g->page_size != 32 && g->page_size != 64)
         return fail(VX_ERR_UNSUPPORTED, "page_size %d not built (16, 32, 64)", g->page_size);
+    if (g->batch > 4096) return fail(VX_ERR_UNSUPPORTED, "batch %d > 4096 not built", g->batch);
     if (g->mla_shared_kv) {
         if (g->num_kv_heads != 1 || g->head_dim_qk != 576 || g->head_dim_v != 512)
             return fail(VX_ERR_UNSUPPORTED, "MLA geometry must be 1 KV head, head_dim_qk 576, head_dim_v 512");
         if (G > 16) return fail(VX_ERR_UNSUPPORTED, "MLA supports at most 16 query heads (got %d)", G);
+        if (g->page_size % vx::MLA_TILE_TOKENS)
+            return fail(VX_ERR_UNSUPPORTED, "MLA page_size must be 32 or 64 (got %d)", g->page_size);
     } else {
         if (g->head_dim_qk != g->head_dim_v) return fail(VX_ERR_UNSUPPORTED, "GQA needs head_dim_qk == head_dim_v");
         if (g->head_dim_qk != 64 && g->head_dim_qk != 128)
             return fail(VX_ERR_UNSUPPORTED, "GQA head_dim %d not built (64, 128)", g->head_dim_qk);
         if (G > 16) return fail(VX_ERR_UNSUPPORTED, "GQA group size %d > 16 not built", G);
-        if (g->num_kv_heads * g->head_dim_qk > 1024)
-            return fail(VX_ERR_UNSUPPORTED, "num_kv_heads * head_dim %d > 1024 not built",
-                        g->num_kv_heads * g->head_dim_qk);
+        const int hkv = g->num_kv_heads;
+        if (hkv > 16 || (hkv & (hkv - 1)))
+            return fail(VX_ERR_UNSUPPORTED, "GQA num_kv_heads %d not built (a power of two <= 16)", hkv);
     }
     return VX_OK;
 }
@@ -133,7 +136,7 @@ vx_status plan(const vx_geometry *g, int32_t k, int32_t num_splits, Plan *p) {
     p->mla = g->mla_shared_kv != 0;
     p->G = g->num_q_heads / g->num_kv_heads;
     p->rows = (int64_t)g->batch * g->num_kv_heads;
-    p->tiles_per_page = g->page_size / vx::DEC_TILE;
+    p->tiles_per_page = g->page_size / (p->mla ? vx::MLA_TILE_TOKENS : vx::DEC_TILE);
     p->units_per_row = (int64_t)k * p->tiles_per_page;
     p->units = p->rows * p->units_per_row;
     int64_t w = num_splits;
@@ -239,7 +242,7 @@ vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q,
     cudaError_t e;
     if (p.mla) {
         CUtensorMap tmK;
-        VX_TRY(make_cache_map(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::DEC_TILE));
+        VX_TRY(make_cache_map(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::MLA_TILE_TOKENS));
         e = vx::launch_decode_mla(a, tmK, p.grid, s, pdl);
     } else {
         CUtensorMap tmK, tmV;

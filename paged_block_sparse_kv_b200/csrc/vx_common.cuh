@@ -72,12 +72,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for phase `parity` of the barrier to complete, for at most WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, unsigned parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for phase `parity` of the barrier to complete, for at most about WAIT_LIMIT_NS.
+// Short waits spin on the non-blocking test_wait (a data tile usually lands within a
+// microsecond); longer ones fall back to try_wait, which may suspend the thread, and
+// read the (slow) global timer only every 1024 tries.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, unsigned parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+    for (int i = 0; i < 4096; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 1024; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
     }
 }

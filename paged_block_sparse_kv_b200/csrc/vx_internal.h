@@ -23,7 +23,8 @@ constexpr int TOPK_SMEM_KEYS = 12288;    // rows up to this many pages keep thei
 constexpr int APPROX_BITS = 12;          // approximate top-k remap width
 constexpr int DEC_WARPS = 8;             // GQA decode: worker warps per block
 constexpr int DEC_STAGES = 3;            // GQA decode: 16-token tiles in flight per warp
-constexpr int DEC_TILE = 16;             // tokens per tile (one mma M or K step)
+constexpr int DEC_TILE = 16;             // GQA decode: tokens per tile (one mma M or K step)
+constexpr int MLA_TILE_TOKENS = 32;      // MLA decode: tokens per tile
 
 // ------------------------------------------------------------------ argument blocks
 struct TableArgs {

@@ -68,6 +68,8 @@ FAKE = 4096  # an aligned non-NULL address; validation fails before anything der
     (dict(head_dim_qk=96, head_dim_v=96), vx.VX_ERR_UNSUPPORTED),
     (dict(head_dim_v=64), vx.VX_ERR_UNSUPPORTED),
     (dict(num_q_heads=8 * 32), vx.VX_ERR_UNSUPPORTED),
+    (dict(num_q_heads=12, num_kv_heads=3), vx.VX_ERR_UNSUPPORTED),
+    (dict(num_q_heads=32, num_kv_heads=32), vx.VX_ERR_UNSUPPORTED),
     (dict(mla_shared_kv=1), vx.VX_ERR_UNSUPPORTED),
     (dict(mla_shared_kv=1, num_kv_heads=1, num_q_heads=32, head_dim_qk=576, head_dim_v=512, page_size=64),
      vx.VX_ERR_UNSUPPORTED),
