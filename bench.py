@@ -329,9 +329,15 @@ def run_vx(args, rank, world, local_rank):
         def topk_only(c):
             vx.vx_topk_pages(c["geo"], c["tab"], c["scores"], k, c["sel"], mode=mode, seed=0, err=c["err"])
 
+        def chain(c):  # the same step as three separate calls (no programmatic dependent launch)
+            score_only(c)
+            topk_only(c)
+            decode_only(c)
+
         nb = max(len(st), min(args.steps, 1000))
         breakdown = {}
-        for name, fn in (("score", score_only), ("topk", topk_only), ("decode_merge", decode_only)):
+        for name, fn in (("score", score_only), ("topk", topk_only), ("decode_merge", decode_only),
+                         ("chain", chain)):
             ms_b, _ = timed_replay(fn, nb, 3)
             breakdown[name + "_us"] = round(ms_b / nb * 1e3, 3)
         if spec.steps:

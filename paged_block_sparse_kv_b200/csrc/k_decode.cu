@@ -87,7 +87,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
                                                   DEC_WARPS * DEC_STAGES * 8) +
                      warp * DEC_STAGES;
 
-    pdl_launch_dependents();
     if (lane == 0) {
         for (int s = 0; s < DEC_STAGES; ++s) mbar_init(bar0 + 8u * s, 1);
         fence_mbar_init();

@@ -97,7 +97,6 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
     const int g4 = lane >> 2, q4 = lane & 3;
     const int mi = lane >> 3, rr = lane & 7;
 
-    pdl_launch_dependents();
     const int64_t c = blockIdx.x;
     if (c >= a.chunks) return;
     const int64_t u_begin = chunk_start(c, a.units, a.chunks);
@@ -205,7 +204,8 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
             }
         }
     };
-    auto start_row = [&](int64_t r) {
+    int64_t q_row = -1;  // row whose Q is staged in shared memory
+    auto stage_q = [&](int64_t r) {
         // stage Q[16 heads][576] into shared memory in the swizzled box layout
         __syncthreads();  // nobody still reads the previous row's Q
         const __nv_bfloat16 *qb = a.q + (size_t)r * a.Hq * MLA_DQK;
@@ -219,6 +219,10 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
                          : "memory");
         }
         __syncthreads();
+        q_row = r;
+    };
+    auto start_row = [&](int64_t r) {
+        if (r != q_row) stage_q(r);
 #pragma unroll
         for (int nt = 0; nt < MLA_NT_PER_WARP; ++nt)
 #pragma unroll
@@ -226,6 +230,10 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
         m_run[0] = m_run[1] = -INFINITY;
         l_run[0] = l_run[1] = 0.f;
     };
+
+    // stage the first row's Q while the first tiles are in flight
+    __syncthreads();  // the producer's first stage meta is visible
+    if (sh.meta[0].row >= 0) stage_q(sh.meta[0].row);
 
     bool failed = false;
     for (uint32_t it = 0;; ++it) {

@@ -71,7 +71,6 @@ __device__ __forceinline__ int score_block_scan(int v, int *tmp, int &total) {
 
 template <int D>
 __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a) {
-    pdl_launch_dependents();
     pdl_wait();  // q, the table and the centroids may come from the previous kernel
     using SP = ScoreSplit<D>;
     constexpr int DPL = SP::DPL, S = SP::S, NCH = SP::NCH;
@@ -237,6 +236,10 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         }
         if (consumed == issued) break;
         const int st = static_cast<int>(consumed % SCORE_STAGES);
+        if (cur_b < 0) {  // first stage: fetch its request's query while the rows are in flight
+            cur_b = meta[st].b;
+            load_query(cur_b);
+        }
         const bool ok = __all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / SCORE_STAGES) & 1u));
         if (!ok) {
             failed = true;

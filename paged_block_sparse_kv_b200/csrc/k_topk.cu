@@ -100,7 +100,6 @@ __device__ __forceinline__ void block_find_bin(TopkShared &sh, int bins, int nee
 
 template <bool APPROX, int THREADS>
 __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
-    pdl_launch_dependents();
     pdl_wait();  // the scores are written by the previous kernel
     __shared__ TopkShared sh;
     extern __shared__ uint32_t skeys[];  // a.smem_keys entries

@@ -39,10 +39,10 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 
 // ------------------------------------------------------------------- PDL
 
-// Let the next kernel on the stream start its prologue now.
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
+// Kernels launched with programmatic dependent launch do not trigger their dependents
+// early: a dependent grid that becomes resident while this one still runs only holds SM
+// resources it cannot use yet (measured slower).  The implicit trigger at block exit still
+// lets the next grid launch as this one drains.
 // Wait until the previous kernel on the stream has finished and its writes are visible.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
