@@ -111,14 +111,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     int64_t cur_row = -1;
     int64_t flushed_to = row_first - 1;  // rows <= flushed_to have their partial written
 
-    auto write_empty = [&](int64_t r) {
-        if (lane < a.G) {
-            float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
-            ml[0] = -INFINITY;
-            ml[1] = 0.f;
-        }
-    };
-    auto flush = [&](int64_t r) {
+    // partial of row `r` (at least one tile attended) for this chunk: slot r + c
+    auto write_partial = [&](int64_t r) {
+        const int64_t slot = r + c;
         float lt[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -130,7 +125,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
                 v += __shfl_xor_sync(FULL, v, 16);
                 lt[nt][i] = v;
             }
-        const int64_t slot = r + c;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -153,6 +147,13 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
                         ml[1] = lt[nt][i];
                     }
                 }
+        }
+    };
+    auto empty_partial = [&](int64_t r) {
+        if (lane < a.G) {
+            float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
+            ml[0] = -INFINITY;
+            ml[1] = 0.f;
         }
     };
     auto start_row = [&](int64_t r) {
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 
     for (;;) {
         // issue loads until the ring is full or the chunk is exhausted
-        while (issued - consumed < DEC_STAGES) {
+        while (!failed && issued - consumed < DEC_STAGES) {
             if (pending == 0) {
                 batch += 32;
                 if (batch >= u_end) break;
@@ -224,24 +225,33 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             __syncwarp();
             ++issued;
         }
-        if (consumed == issued) break;
-
-        const int st = static_cast<int>(consumed % DEC_STAGES);
-        const uint32_t bar = bar0 + 8u * st;
-        const bool ok = __all_sync(FULL, mbar_wait_bounded(bar, (consumed / DEC_STAGES) & 1u));
-        if (!ok) {
-            failed = true;
-            break;
+        // next tile (or the end of the chunk: row = row_last + 1)
+        int64_t row = row_last + 1;
+        int nvalid = 0;
+        int st = 0;
+        if (!failed && consumed != issued) {
+            st = static_cast<int>(consumed % DEC_STAGES);
+            if (!__all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
+                // a load did not arrive in time: report, let every issued load land and
+                // finish the remaining rows as empty
+                if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
+                for (uint32_t i = consumed; i < issued; ++i)
+                    (void)mbar_wait_bounded(bar0 + 8u * (i % DEC_STAGES), (i / DEC_STAGES) & 1u);
+                failed = true;
+                cur_row = -1;
+            } else {
+                row = meta[st].row;
+                nvalid = meta[st].nvalid;
+            }
         }
-        const int64_t row = meta[st].row;
-        const int nvalid = meta[st].nvalid;
         if (row != cur_row) {
             if (cur_row >= 0) {
-                flush(cur_row);
+                write_partial(cur_row);
                 flushed_to = cur_row;
             }
-            for (int64_t r = flushed_to + 1; r < row; ++r) write_empty(r);
+            for (int64_t r = flushed_to + 1; r < row; ++r) empty_partial(r);
             flushed_to = row - 1;
+            if (row > row_last) break;
             start_row(row);
             cur_row = row;
         }
@@ -306,14 +316,14 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             const int tok = rr + 8 * (mi >> 1);
             const bool tail = nvalid < DEC_TILE;
             const int t_lo = 2 * q4, t_hi = 8 + 2 * q4;  // tokens of this lane's A halves
+            const uint32_t mlo = (t_lo < nvalid ? 0x0000ffffu : 0u) | (t_lo + 1 < nvalid ? 0xffff0000u : 0u);
+            const uint32_t mhi = (t_hi < nvalid ? 0x0000ffffu : 0u) | (t_hi + 1 < nvalid ? 0xffff0000u : 0u);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int chunk = (mt & 3) * 2 + (mi & 1);
                 uint32_t v0, v1, v2, v3;
                 ldsm_x4_t(sV + (mt >> 2) * BOX_BYTES + swz128(tok, chunk), v0, v1, v2, v3);
                 if (tail) {
-                    const uint32_t mlo = (t_lo < nvalid ? 0x0000ffffu : 0u) | (t_lo + 1 < nvalid ? 0xffff0000u : 0u);
-                    const uint32_t mhi = (t_hi < nvalid ? 0x0000ffffu : 0u) | (t_hi + 1 < nvalid ? 0xffff0000u : 0u);
                     v0 &= mlo;
                     v1 &= mlo;
                     v2 &= mhi;
@@ -326,20 +336,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         __syncwarp();  // every lane is done with this stage before it is refilled
         ++consumed;
     }
-
-    if (failed) {
-        // a load did not arrive in time: report, let every issued load land, write no partial
-        if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
-        for (uint32_t i = consumed; i < issued; ++i)
-            (void)mbar_wait_bounded(bar0 + 8u * (i % DEC_STAGES), (i / DEC_STAGES) & 1u);
-        for (int64_t r = row_first; r <= row_last; ++r) write_empty(r);
-        return;
-    }
-    if (cur_row >= 0) {
-        flush(cur_row);
-        flushed_to = cur_row;
-    }
-    for (int64_t r = flushed_to + 1; r <= row_last; ++r) write_empty(r);
 }
 
 // Merge: one warp per (row, query head of the group, slice of MERGE_DIMS output dims).

@@ -171,7 +171,7 @@ WsLayout ws_layout(const vx_geometry *g, int32_t max_pages, int32_t k, const Pla
     return l;
 }
 
-// bytes vx_sparse_decode uses: the split partials only (they sit at the start of the layout)
+// bytes vx_sparse_decode uses: the split partials (the start of the layout)
 size_t decode_ws_bytes(const WsLayout &l) { return l.scores; }
 
 // ------------------------------------------------------------------ TMA descriptors
