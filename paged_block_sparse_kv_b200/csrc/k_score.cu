@@ -148,22 +148,63 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         return id;
     };
 
-    // summed query of request b for this lane's head and segment, in the lane's chunk order
+    // summed query of request b for this lane's head and segment, in the lane's chunk order.
+    // The pps lanes that share a (head, segment) split the G query heads of the group
+    // between them (lane of page slot d takes heads d, d + pps, ...), issue all their loads
+    // before using any, and combine with an xor butterfly over the page slots (in plain
+    // chunk order, so every copy ends with the same bits and the sum order is fixed); a
+    // barrel shifter then rotates the chunks into the lane's order.
     float qreg[NCH][8];
     auto load_query = [&](int b) {
         const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)my_head * a.G) * D + my_seg * DPL;
+        bool live[NCH];
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
-            const int ch = (c + lane) % NCH;  // rotated chunk order
+            live[c] = my_seg * DPL + c * 8 < a.score_dims;
 #pragma unroll
             for (int i = 0; i < 8; ++i) qreg[c][i] = 0.f;
-            if (my_seg * DPL + ch * 8 < a.score_dims) {
-                for (int g = 0; g < a.G; ++g) {
-                    float f[8];
-                    bf16x8_to_f32(ld_nc_v4(qb + (size_t)g * D + ch * 8), f);
+        }
+        for (int g0 = my_page; g0 < a.G; g0 += 2 * pps) {
+            const int g1 = g0 + pps;
+            uint4 v0[NCH], v1[NCH];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
-                }
+            for (int c = 0; c < NCH; ++c) {
+                v0[c] = live[c] ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g0 * D + c * 8))
+                                : make_uint4(0u, 0u, 0u, 0u);
+                v1[c] = (live[c] && g1 < a.G) ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g1 * D + c * 8))
+                                              : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                float f[8];
+                bf16x8_to_f32(v0[c], f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
+                bf16x8_to_f32(v1[c], f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
+            }
+        }
+        for (int off = lanes_per_page; off < 32; off <<= 1) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qreg[c][i] += __shfl_xor_sync(FULL, qreg[c][i], off);
+        }
+        // rotate: qreg[c] <- chunk (c + lane) % NCH
+        const int rot = lane % NCH;
+#pragma unroll
+        for (int sh = 1; sh < NCH; sh <<= 1) {
+            if (rot & sh) {
+                float t[NCH][8];
+#pragma unroll
+                for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) t[c][i] = qreg[(c + sh) % NCH][i];
+#pragma unroll
+                for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) qreg[c][i] = t[c][i];
             }
         }
     };

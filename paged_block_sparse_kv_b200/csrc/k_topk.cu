@@ -98,6 +98,26 @@ __device__ __forceinline__ void block_find_bin(TopkShared &sh, int bins, int nee
     __syncthreads();
 }
 
+// One sweep over a row of n scores: every thread issues TOPK_SWEEP_UNROLL loads before it
+// uses any of them, then calls f(j, score) for each.
+constexpr int TOPK_SWEEP_UNROLL = 8;
+template <int THREADS, class F>
+__device__ __forceinline__ void sweep_row(const float *row, int n, F &&f) {
+    for (int j0 = 0; j0 < n; j0 += THREADS * TOPK_SWEEP_UNROLL) {
+        float v[TOPK_SWEEP_UNROLL];
+#pragma unroll
+        for (int i = 0; i < TOPK_SWEEP_UNROLL; ++i) {
+            const int j = j0 + i * THREADS + (int)threadIdx.x;
+            v[i] = j < n ? row[j] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < TOPK_SWEEP_UNROLL; ++i) {
+            const int j = j0 + i * THREADS + (int)threadIdx.x;
+            if (j < n) f(j, v[i]);
+        }
+    }
+}
+
 template <bool APPROX, int THREADS>
 __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
     pdl_wait();  // the scores are written by the previous kernel
@@ -132,21 +152,29 @@ __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
     bool flat = false;
 
     if constexpr (!APPROX) {
-        if (in_smem)
-            for (int j = tid; j < n; j += THREADS) skeys[j] = order_key(row[j]);
+        // first sweep: keys to shared memory and the histogram of the top digit
+        for (int i = tid; i < 2048; i += THREADS) sh.hist[i] = 0;
+        __syncthreads();
+        sweep_row<THREADS>(row, n, [&](int j, float v) {
+            const uint32_t key = order_key(v);
+            if (in_smem) skeys[j] = key;
+            atomicAdd(&sh.hist[key >> 21], 1);
+        });
         __syncthreads();
 #pragma unroll
         for (int pass = 0; pass < 3; ++pass) {
             const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
             const int bins = pass == 2 ? 1024 : 2048;
             const uint32_t dmask = (uint32_t)bins - 1u;
-            for (int i = tid; i < bins; i += THREADS) sh.hist[i] = 0;
-            __syncthreads();
-            for (int j = tid; j < n; j += THREADS) {
-                const uint32_t key = in_smem ? skeys[j] : order_key(row[j]);
-                if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & dmask], 1);
+            if (pass > 0) {
+                for (int i = tid; i < bins; i += THREADS) sh.hist[i] = 0;
+                __syncthreads();
+                for (int j = tid; j < n; j += THREADS) {
+                    const uint32_t key = in_smem ? skeys[j] : order_key(row[j]);
+                    if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & dmask], 1);
+                }
+                __syncthreads();
             }
-            __syncthreads();
             block_find_bin<THREADS>(sh, bins, remaining);
             const int digit = sh.bcast[0], above = sh.bcast[1], cnt = sh.bcast[2];
             remaining -= above;
@@ -157,12 +185,13 @@ __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
         }
     } else {
         // row min / max
+        // first sweep: min / max, raw scores staged in shared memory
         float mn = INFINITY, mx = -INFINITY;
-        for (int j = tid; j < n; j += THREADS) {
-            const float s = row[j];
-            mn = fminf(mn, s);
-            mx = fmaxf(mx, s);
-        }
+        sweep_row<THREADS>(row, n, [&](int j, float v) {
+            if (in_smem) skeys[j] = __float_as_uint(v);
+            mn = fminf(mn, v);
+            mx = fmaxf(mx, v);
+        });
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(FULL, mn, off));
@@ -184,10 +213,11 @@ __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
         const float range = __fsub_rn(mx, mn);
         scale = __fdiv_rn(static_cast<float>(TOPK_HIST), range);
         flat = !(mx > mn) || isinf(scale);
-        for (int j = tid; j < n; j += THREADS) {
+        for (int j = tid; j < n; j += THREADS) {  // each thread rereads only what it staged
             uint32_t code = 0;
             if (!flat) {
-                const float f = floorf(__fmul_rn(__fsub_rn(row[j], lo), scale));
+                const float v = in_smem ? __uint_as_float(skeys[j]) : row[j];
+                const float f = floorf(__fmul_rn(__fsub_rn(v, lo), scale));
                 code = f >= float(TOPK_HIST - 1) ? TOPK_HIST - 1 : static_cast<uint32_t>(f);
             }
             if (in_smem) skeys[j] = code;
