@@ -54,6 +54,7 @@ __device__ __forceinline__ void centroid_warp(const __nv_bfloat16 *__restrict__ 
         double acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+#pragma unroll 4
         for (int t = lane / CPR; t < m; t += RPL) {
             const void *src = (t == alt_slot) ? static_cast<const void *>(alt + chunk * 8)
                                               : static_cast<const void *>(rows + (size_t)t * D + chunk * 8);
@@ -82,6 +83,7 @@ __device__ __forceinline__ void centroid_warp(const __nv_bfloat16 *__restrict__ 
             double acc[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+#pragma unroll 8
             for (int t = 0; t < m; ++t) {
                 const void *src = (t == alt_slot) ? static_cast<const void *>(alt + chunk * 8)
                                                   : static_cast<const void *>(rows + (size_t)t * D + chunk * 8);

@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
                 meta[st].nvalid = nv;
                 const uint32_t bar = bar0 + 8u * st;
                 const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
-                fence_proxy_async_smem();  // earlier generic reads of this stage come first
+                // no proxy fence: this stage's earlier shared-memory reads have completed,
+                // their values were consumed before the __syncwarp that released the stage
                 mbar_arrive_expect_tx(bar, STAGE_BYTES);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
@@ -341,9 +342,10 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 // Merge: one warp per (row, query head of the group, slice of MERGE_DIMS output dims).
 // The row's partials are those of the chunks c_lo..c_hi that touch it (slot row + c).
 // Lanes first read every partial's (max, sum) in parallel to form the common max and the
-// total; the weighted outputs are then accumulated MERGE_UNROLL partials at a time, each
-// lane owning MERGE_DIMS/32 dims of the slice.
-constexpr int MERGE_UNROLL = 4;
+// total (lane i keeps partial i's weight); the weighted outputs are then accumulated
+// MERGE_UNROLL partials at a time, each lane owning MERGE_DIMS/32 dims of the slice, with
+// all of a group's loads issued before any is used.
+constexpr int MERGE_UNROLL = 8;
 constexpr int MERGE_DIMS = 128;
 
 template <int DV>
@@ -364,9 +366,14 @@ __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     const int np = static_cast<int>(c_hi - c_lo + 1);
     const float *ml0 = a.ml_part + ((r + c_lo) * a.G + g) * 2;                    // partial i at + i*G*2
     const float *o0 = a.o_part + ((r + c_lo) * a.G + g) * DV + slice * SLICE;      // partial i at + i*G*DV
-    // common max and total over all partials (lane i handles partials i, i + 32, ...)
-    float M = -INFINITY;
-    for (int i = lane; i < np; i += 32) M = fmaxf(M, ml0[(int64_t)i * a.G * 2]);
+    // common max and total over all partials (lane i handles partials i, i + 32, ...);
+    // lane i < 32 keeps partial i's weight for the accumulation below
+    float M = -INFINITY, m_mine = -INFINITY;
+    for (int i = lane; i < np; i += 32) {
+        const float m = ml0[(int64_t)i * a.G * 2];
+        if (i < 32) m_mine = m;
+        M = fmaxf(M, m);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
     float lsum = 0.f;
@@ -377,6 +384,7 @@ __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
         }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(FULL, lsum, off);
+    const float w_mine = (M == -INFINITY || m_mine == -INFINITY) ? 0.f : exp2f(m_mine - M);
 
     constexpr int PER = SLICE / 32;  // dims per lane
     float o[PER];
@@ -384,25 +392,31 @@ __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     for (int i = 0; i < PER; ++i) o[i] = 0.f;
     if (M != -INFINITY) {
         for (int i0 = 0; i0 < np; i0 += MERGE_UNROLL) {
-            float w[MERGE_UNROLL];
+            // loads first (an empty partial holds no output values: read, then dropped)
             float2 v[MERGE_UNROLL][PER / 2];
 #pragma unroll
             for (int u = 0; u < MERGE_UNROLL; ++u) {
                 const int i = i0 + u;
-                const float m = i < np ? ml0[(int64_t)i * a.G * 2] : -INFINITY;
-                w[u] = m == -INFINITY ? 0.f : exp2f(m - M);
                 const float *op = o0 + (int64_t)i * a.G * DV + lane * PER;
 #pragma unroll
                 for (int d = 0; d < PER / 2; ++d)
-                    v[u][d] = w[u] != 0.f ? *reinterpret_cast<const float2 *>(op + 2 * d) : make_float2(0.f, 0.f);
+                    v[u][d] = i < np ? *reinterpret_cast<const float2 *>(op + 2 * d) : make_float2(0.f, 0.f);
             }
 #pragma unroll
-            for (int u = 0; u < MERGE_UNROLL; ++u)
+            for (int u = 0; u < MERGE_UNROLL; ++u) {
+                const int i = i0 + u;
+                float w = __shfl_sync(FULL, w_mine, i & 31);
+                if (i >= 32) {  // beyond the lanes' cache: reread (m)
+                    const float m = i < np ? ml0[(int64_t)i * a.G * 2] : -INFINITY;
+                    w = m == -INFINITY ? 0.f : exp2f(m - M);
+                }
+                if (i >= np) w = 0.f;
 #pragma unroll
                 for (int d = 0; d < PER / 2; ++d) {
-                    o[2 * d] += w[u] * v[u][d].x;
-                    o[2 * d + 1] += w[u] * v[u][d].y;
+                    o[2 * d] += w != 0.f ? w * v[u][d].x : 0.f;
+                    o[2 * d + 1] += w != 0.f ? w * v[u][d].y : 0.f;
                 }
+            }
         }
     }
     const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);

@@ -149,7 +149,8 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
         if (lane == 0) {
             sh.meta[st].row = row;
             sh.meta[st].nvalid = nv;
-            fence_proxy_async_smem();
+            // no proxy fence: this stage's earlier shared-memory reads have completed,
+            // their values were consumed before the barrier that released the stage
             mbar_arrive_expect_tx(bar, MLA_TILE);
             const uint32_t dst = sK0 + (uint32_t)st * MLA_TILE;
 #pragma unroll
@@ -209,13 +210,23 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
         // stage Q[16 heads][576] into shared memory in the swizzled box layout
         __syncthreads();  // nobody still reads the previous row's Q
         const __nv_bfloat16 *qb = a.q + (size_t)r * a.Hq * MLA_DQK;
-        for (int i = tid; i < 16 * (MLA_DQK / 8); i += MLA_THREADS) {
+        constexpr int QCH = 16 * (MLA_DQK / 8) / MLA_THREADS;  // 16-byte chunks per thread
+        static_assert(16 * (MLA_DQK / 8) % MLA_THREADS == 0, "Q chunks split evenly");
+        uint4 v[QCH];  // every load is issued before the first store
+#pragma unroll
+        for (int k = 0; k < QCH; ++k) {
+            const int i = tid + k * MLA_THREADS;
             const int head = i / (MLA_DQK / 8), ch = i % (MLA_DQK / 8);
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (head < a.G) v = *reinterpret_cast<const uint4 *>(qb + (size_t)head * MLA_DQK + ch * 8);
+            v[k] = head < a.G ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)head * MLA_DQK + ch * 8))
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < QCH; ++k) {
+            const int i = tid + k * MLA_THREADS;
+            const int head = i / (MLA_DQK / 8), ch = i % (MLA_DQK / 8);
             const uint32_t dst = sQ + (ch >> 3) * MLA_QBOX + swz128(head, ch & 7);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
-                         "r"(v.w)
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k].x), "r"(v[k].y),
+                         "r"(v[k].z), "r"(v[k].w)
                          : "memory");
         }
         __syncthreads();

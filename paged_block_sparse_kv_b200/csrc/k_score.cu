@@ -267,9 +267,10 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
                 mbar_arrive_expect_tx(bar, (uint32_t)n * row_bytes);  // all bytes announced first
             }
             __syncwarp();
+            // no proxy fence: this stage's earlier shared-memory reads have completed, their
+            // values were consumed before the __syncwarp that released the stage
             if ((take >> lane) & 1u) {
                 const uint32_t slot = __popc(take & ((1u << lane) - 1u));
-                fence_proxy_async_smem();  // earlier generic reads of this stage come first
                 bulk_load(dst + slot * row_bytes, a.centroids + (size_t)my_id * a.Hkv * D, row_bytes, bar);
             }
             __syncwarp();

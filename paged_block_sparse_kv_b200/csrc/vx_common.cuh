@@ -155,13 +155,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // ------------------------------------------------------------------- loads
 
-__device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
+// 16-byte read-only load; an intrinsic rather than volatile asm so the compiler may issue
+// several before the first is used.
+__device__ __forceinline__ uint4 ld_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 // 8 bf16 packed in a uint4 -> 8 floats (exact widening)
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
