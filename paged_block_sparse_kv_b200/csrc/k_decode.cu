@@ -24,6 +24,8 @@
 // n-tile), online softmax in base 2, P^T moved into the B-operand layout with
 // movmatrix, O^T += V^T P^T with ldmatrix.trans for V.  Value rows past the request's
 // length are zeroed in registers, so NaN in unused slots cannot leak.
+#include <type_traits>
+
 #include "vx_internal.h"
 
 namespace vx {
@@ -101,8 +103,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     const int64_t u_end = chunk_start(c + 1, a.units, a.chunks);
     const int64_t row_first = u_begin / a.units_per_row;
     const int64_t row_last = (u_end - 1) / a.units_per_row;
-
-    pdl_wait();  // the selection comes from the previous kernel
 
     // ---- per-row state
     uint32_t qf[NT][MT][2];
@@ -184,6 +184,14 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             }
         }
     };
+
+    // The first row's query is read before waiting on the previous kernel: the query is an
+    // input of the call, complete before this grid starts (the grid runs either in plain
+    // stream order or after the top-k kernel, which itself starts after the scorer ends).
+    // Only the selection is written by the previous kernel.
+    start_row(row_first);
+    cur_row = row_first;
+    pdl_wait();
 
     // ---- pipeline
     int64_t batch = u_begin;
@@ -339,20 +347,21 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     }
 }
 
-// Merge: one warp per (row, query head of the group, slice of MERGE_DIMS output dims).
-// The row's partials are those of the chunks c_lo..c_hi that touch it (slot row + c).
-// Lanes first read every partial's (max, sum) in parallel to form the common max and the
-// total (lane i keeps partial i's weight); the weighted outputs are then accumulated
-// MERGE_UNROLL partials at a time, each lane owning MERGE_DIMS/32 dims of the slice, with
-// all of a group's loads issued before any is used.
-constexpr int MERGE_UNROLL = 8;
-constexpr int MERGE_DIMS = 128;
-
-template <int DV>
+// Merge: one warp per (row, query head of the group, slice of 32*PER output dims), PER
+// consecutive dims per lane.  The row's partials are those of the chunks c_lo..c_hi that
+// touch it (slot row + c).  Partials are taken GROUP at a time: every lane reads its dims
+// of GROUP outputs, and lane i reads partial i's (max, sum), all loads issued before any
+// is used, so a row with up to GROUP partials costs one round trip.  The common max comes
+// first (over all partials), then the weighted outputs are summed in partial order.  The
+// launcher picks PER = 1 (more warps, for few rows with many partials) or a wider slice
+// (fewer warps, for many rows with few partials).
+template <int DV, int PER, int GROUP>
 __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     pdl_wait();
-    constexpr int SLICE = DV < MERGE_DIMS ? DV : MERGE_DIMS;
+    constexpr int SLICE = 32 * PER;
     constexpr int NSLICE = DV / SLICE;
+    static_assert(DV % SLICE == 0 && GROUP <= 32, "merge shape");
+    using VecT = typename std::conditional<PER == 4, float4, typename std::conditional<PER == 2, float2, float>::type>::type;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t item = (int64_t)blockIdx.x * 8 + warp;
     const int64_t rows = (int64_t)a.B * a.Hkv;
@@ -364,68 +373,73 @@ __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     const int64_t c_lo = chunk_of(r * a.units_per_row, a.units, a.chunks);
     const int64_t c_hi = chunk_of((r + 1) * a.units_per_row - 1, a.units, a.chunks);
     const int np = static_cast<int>(c_hi - c_lo + 1);
-    const float *ml0 = a.ml_part + ((r + c_lo) * a.G + g) * 2;                    // partial i at + i*G*2
-    const float *o0 = a.o_part + ((r + c_lo) * a.G + g) * DV + slice * SLICE;      // partial i at + i*G*DV
-    // common max and total over all partials (lane i handles partials i, i + 32, ...);
-    // lane i < 32 keeps partial i's weight for the accumulation below
-    float M = -INFINITY, m_mine = -INFINITY;
-    for (int i = lane; i < np; i += 32) {
-        const float m = ml0[(int64_t)i * a.G * 2];
-        if (i < 32) m_mine = m;
-        M = fmaxf(M, m);
-    }
+    const float *ml0 = a.ml_part + ((r + c_lo) * a.G + g) * 2;                               // partial i at + i*G*2
+    const float *o0 = a.o_part + ((r + c_lo) * a.G + g) * DV + slice * SLICE + lane * PER;   // partial i at + i*G*DV
+
+    auto load_o = [&](int i) -> VecT {
+        VecT z;
+        memset(&z, 0, sizeof(z));
+        return i < np ? *reinterpret_cast<const VecT *>(o0 + (int64_t)i * a.G * DV) : z;
+    };
+    // first group's outputs and (max, sum), loaded together
+    VecT v[GROUP];
+#pragma unroll
+    for (int u = 0; u < GROUP; ++u) v[u] = load_o(u);
+    const float m_first = lane < np ? ml0[(int64_t)lane * a.G * 2] : -INFINITY;
+    const float l_first = lane < np ? ml0[(int64_t)lane * a.G * 2 + 1] : 0.f;
+
+    // common max and total over all partials (lane i handles partials i, i + 32, ...)
+    float M = m_first;
+    for (int i = lane + 32; i < np; i += 32) M = fmaxf(M, ml0[(int64_t)i * a.G * 2]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
     float lsum = 0.f;
-    if (M != -INFINITY)
-        for (int i = lane; i < np; i += 32) {
+    if (M != -INFINITY) {
+        if (m_first != -INFINITY) lsum = exp2f(m_first - M) * l_first;
+        for (int i = lane + 32; i < np; i += 32) {
             const float m = ml0[(int64_t)i * a.G * 2];
             if (m != -INFINITY) lsum += exp2f(m - M) * ml0[(int64_t)i * a.G * 2 + 1];
         }
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(FULL, lsum, off);
-    const float w_mine = (M == -INFINITY || m_mine == -INFINITY) ? 0.f : exp2f(m_mine - M);
+    // lane i keeps the weight of partial i of the first group
+    const float w_first = (M == -INFINITY || m_first == -INFINITY) ? 0.f : exp2f(m_first - M);
 
-    constexpr int PER = SLICE / 32;  // dims per lane
     float o[PER];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) o[i] = 0.f;
+    for (int d = 0; d < PER; ++d) o[d] = 0.f;
+    // an empty partial (max -inf) holds no output values: read, then dropped
+    auto add = [&](const VecT &x, float w) {
+        const float *xv = reinterpret_cast<const float *>(&x);
+#pragma unroll
+        for (int d = 0; d < PER; ++d) o[d] += w != 0.f ? w * xv[d] : 0.f;
+    };
     if (M != -INFINITY) {
-        for (int i0 = 0; i0 < np; i0 += MERGE_UNROLL) {
-            // loads first (an empty partial holds no output values: read, then dropped)
-            float2 v[MERGE_UNROLL][PER / 2];
 #pragma unroll
-            for (int u = 0; u < MERGE_UNROLL; ++u) {
-                const int i = i0 + u;
-                const float *op = o0 + (int64_t)i * a.G * DV + lane * PER;
+        for (int u = 0; u < GROUP; ++u) add(v[u], __shfl_sync(FULL, w_first, u));
+#pragma unroll 1
+        for (int g0 = GROUP; g0 < np; g0 += GROUP) {  // rows with more than GROUP partials
 #pragma unroll
-                for (int d = 0; d < PER / 2; ++d)
-                    v[u][d] = i < np ? *reinterpret_cast<const float2 *>(op + 2 * d) : make_float2(0.f, 0.f);
-            }
+            for (int u = 0; u < GROUP; ++u) v[u] = load_o(g0 + u);
+            // lane u < GROUP computes the weight of partial g0 + u
+            const int i = g0 + lane;
+            const float m = (lane < GROUP && i < np) ? ml0[(int64_t)i * a.G * 2] : -INFINITY;
+            const float w_lane = m == -INFINITY ? 0.f : exp2f(m - M);
 #pragma unroll
-            for (int u = 0; u < MERGE_UNROLL; ++u) {
-                const int i = i0 + u;
-                float w = __shfl_sync(FULL, w_mine, i & 31);
-                if (i >= 32) {  // beyond the lanes' cache: reread (m)
-                    const float m = i < np ? ml0[(int64_t)i * a.G * 2] : -INFINITY;
-                    w = m == -INFINITY ? 0.f : exp2f(m - M);
-                }
-                if (i >= np) w = 0.f;
-#pragma unroll
-                for (int d = 0; d < PER / 2; ++d) {
-                    o[2 * d] += w != 0.f ? w * v[u][d].x : 0.f;
-                    o[2 * d + 1] += w != 0.f ? w * v[u][d].y : 0.f;
-                }
-            }
+            for (int u = 0; u < GROUP; ++u) add(v[u], __shfl_sync(FULL, w_lane, u));
         }
     }
     const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);
     const size_t head = (size_t)b * a.Hq + (size_t)h * a.G + g;
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
     __nv_bfloat16 *dst = a.out + head * DV + slice * SLICE + lane * PER;
+    if constexpr (PER == 1) {
+        *dst = __float2bfloat16_rn(o[0] * inv);
+    } else {
 #pragma unroll
-    for (int i = 0; i < PER; i += 2)
-        *reinterpret_cast<uint32_t *>(dst + i) = pack_bf16x2(o[i] * inv, o[i + 1] * inv);
+        for (int d = 0; d < PER; d += 2) *reinterpret_cast<uint32_t *>(dst + d) = pack_bf16x2(o[d] * inv, o[d + 1] * inv);
+    }
     if (a.lse && lane == 0 && slice == 0)
         a.lse[head] = lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
 }
@@ -452,14 +466,32 @@ cudaError_t launch_decode_gqa(const DecodeArgs &a, const CUtensorMap &tmK, const
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl) {
-    const int nslice = a.Dv > MERGE_DIMS ? a.Dv / MERGE_DIMS : 1;
-    const int64_t items = (int64_t)a.B * a.Hkv * a.G * nslice;
+template <int DV>
+static cudaError_t launch_merge_dv(const DecodeArgs &a, cudaStream_t s, bool pdl) {
+    constexpr int PW = DV >= 128 ? 4 : 2;  // dims per lane of the wide shape
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)a.B * a.Hkv;
+    const int64_t wide_items = rows * a.G * (DV / (32 * PW));
+    // partials of the row with the most: the chunks it spans
+    const int64_t np_max = (a.units_per_row * a.chunks + a.units - 1) / a.units + 1;
+    if (wide_items >= (int64_t)sms * 8 * 4) {  // enough warps for four per SM slot
+        const dim3 grid((unsigned)((wide_items + 7) / 8));
+        return launch_k(k_merge<DV, PW, 32 / PW>, grid, dim3(256), 0, s, pdl, a);
+    }
+    const int64_t items = rows * a.G * (DV / 32);
     const dim3 grid((unsigned)((items + 7) / 8));
+    if (np_max <= 16) return launch_k(k_merge<DV, 1, 16>, grid, dim3(256), 0, s, pdl, a);
+    return launch_k(k_merge<DV, 1, 32>, grid, dim3(256), 0, s, pdl, a);
+}
+
+cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl) {
     switch (a.Dv) {
-        case 64: return launch_k(k_merge<64>, grid, dim3(256), 0, s, pdl, a);
-        case 128: return launch_k(k_merge<128>, grid, dim3(256), 0, s, pdl, a);
-        case 512: return launch_k(k_merge<512>, grid, dim3(256), 0, s, pdl, a);
+        case 64: return launch_merge_dv<64>(a, s, pdl);
+        case 128: return launch_merge_dv<128>(a, s, pdl);
+        case 512: return launch_merge_dv<512>(a, s, pdl);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -109,7 +109,40 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
         tma_prefetch_desc(&tmK);
     }
     __syncthreads();
-    pdl_wait();  // the selection comes from the previous kernel
+
+    int64_t q_row = -1;  // row whose Q is staged in shared memory
+    auto stage_q = [&](int64_t r) {
+        // stage Q[16 heads][576] into shared memory in the swizzled box layout
+        __syncthreads();  // nobody still reads the previous row's Q
+        const __nv_bfloat16 *qb = a.q + (size_t)r * a.Hq * MLA_DQK;
+        constexpr int QCH = 16 * (MLA_DQK / 8) / MLA_THREADS;  // 16-byte chunks per thread
+        static_assert(16 * (MLA_DQK / 8) % MLA_THREADS == 0, "Q chunks split evenly");
+        uint4 v[QCH];  // every load is issued before the first store
+#pragma unroll
+        for (int k = 0; k < QCH; ++k) {
+            const int i = tid + k * MLA_THREADS;
+            const int head = i / (MLA_DQK / 8), ch = i % (MLA_DQK / 8);
+            v[k] = head < a.G ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)head * MLA_DQK + ch * 8))
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < QCH; ++k) {
+            const int i = tid + k * MLA_THREADS;
+            const int head = i / (MLA_DQK / 8), ch = i % (MLA_DQK / 8);
+            const uint32_t dst = sQ + (ch >> 3) * MLA_QBOX + swz128(head, ch & 7);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k].x), "r"(v[k].y),
+                         "r"(v[k].z), "r"(v[k].w)
+                         : "memory");
+        }
+        __syncthreads();
+        q_row = r;
+    };
+    // Q of the chunk's first row is staged before waiting on the previous kernel: the query
+    // is an input of the call, complete before this grid starts (the grid runs either in
+    // plain stream order or after the top-k kernel, which itself starts after the scorer
+    // ends).  Only the selection is written by the previous kernel.
+    stage_q(row_first);
+    pdl_wait();
 
     // ---- producer state (warp 0)
     int64_t batch = u_begin;
@@ -205,33 +238,6 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
             }
         }
     };
-    int64_t q_row = -1;  // row whose Q is staged in shared memory
-    auto stage_q = [&](int64_t r) {
-        // stage Q[16 heads][576] into shared memory in the swizzled box layout
-        __syncthreads();  // nobody still reads the previous row's Q
-        const __nv_bfloat16 *qb = a.q + (size_t)r * a.Hq * MLA_DQK;
-        constexpr int QCH = 16 * (MLA_DQK / 8) / MLA_THREADS;  // 16-byte chunks per thread
-        static_assert(16 * (MLA_DQK / 8) % MLA_THREADS == 0, "Q chunks split evenly");
-        uint4 v[QCH];  // every load is issued before the first store
-#pragma unroll
-        for (int k = 0; k < QCH; ++k) {
-            const int i = tid + k * MLA_THREADS;
-            const int head = i / (MLA_DQK / 8), ch = i % (MLA_DQK / 8);
-            v[k] = head < a.G ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)head * MLA_DQK + ch * 8))
-                              : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < QCH; ++k) {
-            const int i = tid + k * MLA_THREADS;
-            const int head = i / (MLA_DQK / 8), ch = i % (MLA_DQK / 8);
-            const uint32_t dst = sQ + (ch >> 3) * MLA_QBOX + swz128(head, ch & 7);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k].x), "r"(v[k].y),
-                         "r"(v[k].z), "r"(v[k].w)
-                         : "memory");
-        }
-        __syncthreads();
-        q_row = r;
-    };
     auto start_row = [&](int64_t r) {
         if (r != q_row) stage_q(r);
 #pragma unroll
@@ -242,9 +248,9 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
         l_run[0] = l_run[1] = 0.f;
     };
 
-    // stage the first row's Q while the first tiles are in flight
+    // the first tile's Q if it is not row_first's (start_row would stage it otherwise)
     __syncthreads();  // the producer's first stage meta is visible
-    if (sh.meta[0].row >= 0) stage_q(sh.meta[0].row);
+    if (sh.meta[0].row >= 0 && sh.meta[0].row != q_row) stage_q(sh.meta[0].row);
 
     bool failed = false;
     for (uint32_t it = 0;; ++it) {

@@ -120,7 +120,6 @@ __device__ __forceinline__ void sweep_row(const float *row, int n, F &&f) {
 
 template <bool APPROX, int THREADS>
 __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
-    pdl_wait();  // the scores are written by the previous kernel
     __shared__ TopkShared sh;
     extern __shared__ uint32_t skeys[];  // a.smem_keys entries
     const int b = blockIdx.y, h = blockIdx.x;
@@ -139,6 +138,10 @@ __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
         for (int i = tid; i < a.k; i += THREADS) out[i] = i < n ? i : -1;
         return;
     }
+    // Everything above reads only inputs of the call, complete before this grid starts (it
+    // runs in plain stream order or after the scorer, which starts in stream order); the
+    // scores come from the previous kernel.
+    pdl_wait();
     const bool in_smem = n <= a.smem_keys;
 
     // per-thread contiguous run [r0, r1) used by the ordered compaction
