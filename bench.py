@@ -37,11 +37,15 @@ DEFAULT_CONFIG = "qwen3_1p7b_gqa_b32"
 
 # DRAM traffic of the dominant kernel from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # as a multiple of the algorithmic bytes of the captured launch; valid only for the kernel source it was
-# taken on (sha256 of the file), otherwise the bench reports null.  Summary: profiles/k_decode_gqa_qwen3_b8.md.
+# taken on (sha256 of the file), otherwise the bench reports null.  Summaries: profiles/k_decode_gqa_*.md,
+# profiles/k_decode_mla_*.md.
 DECODE_TRAFFIC = {
-    "csrc/k_decode.cu": {"sha256": "1027e0aaadb1f87706e92d512b14beaf9b0af86b515cc74e3f90a307889460ff",
-                         "ratio": 68.43 / 67.106, "workload": "qwen3_1p7b_gqa_b32",
+    "csrc/k_decode.cu": {"sha256": "0e3f14d032c0b67f041218ae95b217fde4474ebe1bb1a2ab573b5b9a772fc330",
+                         "ratio": (67.244544 + 1.102592) / 67.097856, "workload": "qwen3_1p7b_gqa_b32",
                          "note": "captured at batch 8 (67.1 MB), scaled to the full launch by its bytes"},
+    "csrc/k_decode_mla.cu": {"sha256": "a7960aede43728c07db8e904853a66658d6d8cb6b19778089bb1b328c8156430",
+                             "ratio": (38.134784 + 0.329472) / 38.264896, "workload": "mla_576_512_b16",
+                             "note": "captured on the full workload (38.3 MB)"},
 }
 
 
@@ -66,6 +70,9 @@ def parse():
     ap.add_argument("--mode", default="exact", choices=["exact", "approx"])
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--batch", type=int, default=0, help="override the batch (small profiling cases only)")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="independent input copies to rotate (0: enough for > 3x L2); fewer only for ncu "
+                         "captures, which flush the caches before each captured launch themselves")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -222,14 +229,17 @@ def run_vx(args, rank, world, local_rank):
         fused(st[0])
         torch.cuda.synchronize()
         total0 = step_bytes(w, st[0]["sel"], w.seq_lens, k)[0]
-        for i in range(1, max(2, math.ceil(3 * L2_BYTES / max(total0, 1)))):
+        # the other copies' bytes between two uses of one copy exceed 3x L2
+        n_copies = args.copies or max(2, math.floor(3 * L2_BYTES / max(total0, 1)) + 2)
+        for i in range(1, n_copies):
             w = synth.make(spec, seed0 + i, dev)
             geo = geom(w)
             tab = vx.PageTable(w.page_ptr, w.page_indices, w.seq_lens, w.max_pages)
             st.append(dict(w=w, geo=geo, tab=tab, cen=rebuild_centroids(w, geo, tab), q=w.q, append=False,
                            seq_lens=w.seq_lens, **buffers(w, geo)))
         launches_per_step = 4
-        l2_note = "inputs rotate over {n} independent copies, {mb:.0f} MB between reuses (> 3x L2)"
+        l2_note = "inputs rotate over {n} independent copies, {mb:.0f} MB between reuses " + (
+            "(> 3x L2)" if (n_copies - 1) * total0 > 3 * L2_BYTES else "(fewer than 3x L2: profiling run only)")
     else:
         # continuous batching: one workload, `steps` consecutive decode steps, each appending
         # one token per request before it decodes (replays rewrite the same slots)
