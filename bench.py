@@ -76,6 +76,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--persistent", action="store_true",
+                    help="time vx_block_topk_decode_persistent (one persistent kernel) instead of the chained call")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time the score, top-k and decode calls separately (CUDA events, graphs)")
     return ap.parse_args()
@@ -201,7 +203,7 @@ def run_vx(args, rank, world, local_rank):
         lse = torch.empty((B, spec.num_q_heads), dtype=torch.float32, device=dev)
         scores = torch.empty((B, spec.num_kv_heads, w.max_pages), dtype=torch.float32, device=dev)
         sel = torch.empty((B, spec.num_kv_heads, k), dtype=torch.int32, device=dev)
-        ws = torch.empty(vx.vx_workspace_size(geo, w.max_pages, k, args.splits), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(vx.vx_workspace_size(geo, w.max_pages, k, args.splits), dtype=torch.uint8, device=dev)
         err = torch.zeros(1, dtype=torch.int32, device=dev)
         return dict(out=out, lse=lse, scores=scores, sel=sel, ws=ws, err=err)
 
@@ -214,6 +216,11 @@ def run_vx(args, rank, world, local_rank):
         if c["append"]:
             vx.vx_centroid_update(c["geo"], c["tab"], c["w"].k_cache, c["cen"], v_cache=c["w"].v_cache,
                                   k_new=c["k_new"], v_new=c["v_new"], err=c["err"])
+        if args.persistent:
+            vx.vx_block_topk_decode_persistent(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"],
+                                               k, c["out"], c["ws"], lse=c["lse"], scores_out=c["scores"],
+                                               sel_out=c["sel"], err=c["err"])
+            return
         vx.vx_block_topk_decode(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"], k, c["out"],
                                 c["ws"], lse=c["lse"], mode=mode, seed=0, num_splits=args.splits,
                                 scores_out=c["scores"], sel_out=c["sel"], err=c["err"])
@@ -409,6 +416,7 @@ def run_vx(args, rank, world, local_rank):
                        "num_kv_heads": spec.num_kv_heads, "head_dim_qk": spec.head_dim_qk,
                        "head_dim_v": spec.head_dim_v, "page_size": spec.page_size, "k_pages": k,
                        "context": list(spec.ctx), "topk_mode": args.mode, "splits": args.splits or "planned",
+                       "entry": "vx_block_topk_decode_persistent" if args.persistent else "vx_block_topk_decode",
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": l2_note.format(n=len(st), mb=mean_bytes * max(1, len(st) - 1) / 1e6)},
             "hbm": {"roofline_bytes_per_step": int(mean_bytes), "achieved_gbs": round(step_gbs, 1),

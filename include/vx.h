@@ -168,7 +168,8 @@ vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, c
  * previous one's tail (paper note, 系统设计 3: fusion of the sequence-local steps and
  * workload planning).  Same arguments and results as the three calls.  scores_out and
  * sel_out (may be NULL) receive the intermediate scores and selection; when NULL they
- * live in the workspace.  score_dims as in vx_score_pages.
+ * live in the workspace.  score_dims as in vx_score_pages.  ws: vx_workspace_size bytes,
+ * no initial contents needed.
  */
 vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *table, const void *q,
                                const void *k_cache, const void *v_cache, const void *centroids,
@@ -176,6 +177,31 @@ vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *tabl
                                int32_t score_dims, int32_t num_splits, void *out, float *lse,
                                float *scores_out, int32_t *sel_out, void *ws, size_t ws_bytes,
                                int32_t *err, void *stream);
+
+/*
+ * The same decode step (exact top-k, full score dims) as ONE persistent kernel (paper note,
+ * 系统设计 3: fusion and workload planning, taken to a single launch).  Its warps take work
+ * items from two ticket counters: score a span of one request's pages, attend a span of
+ * one (request, KV head) row's selected tiles (the row's last span merges the row), and,
+ * in request order, select one row (exact radix top-k on a warp, ties to the lower page).
+ * Every wait is on a smaller ticket or is helped along by the waiting warp, and is bounded
+ * (a timeout sets VX_DATA_TIMEOUT), so the launch always ends.
+ *   Geometry: GQA with head_dim_qk == head_dim_v in {64, 128}, num_kv_heads <= 16, at
+ *   most 16 query heads per KV head, batch <= 1024 (else VX_ERR_UNSUPPORTED).
+ *   Results: the same scores and selection bits as vx_block_topk_decode with mode 0; out
+ *   and lse differ only by rounding (its own split of the attention).
+ *   Speed: slower than vx_block_topk_decode on B200 for the workloads measured here (its
+ *   warp-level selection is the bottleneck); kept for study and as the fused reference.
+ * ws: vx_workspace_size(geo, max_pages, k, 0) bytes.  ZERO-FILL IT ONCE before its first
+ * use here (e.g. cudaMemset after allocating): its first bytes hold the kernel's counters,
+ * which every call leaves zero again.  No other entry point writes them, so one workspace
+ * may serve every call (one call at a time).
+ */
+vx_status vx_block_topk_decode_persistent(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                                          const void *k_cache, const void *v_cache, const void *centroids,
+                                          int32_t k, float sm_scale, void *out, float *lse, float *scores_out,
+                                          int32_t *sel_out, void *ws, size_t ws_bytes, int32_t *err,
+                                          void *stream);
 
 /*
  * vx_sparse_decode without a caller workspace, for callers that cannot allocate device
@@ -209,7 +235,9 @@ vx_status vx_sparse_decode_noalloc(const vx_geometry *geo, const vx_page_table *
 /*
  * Workspace bytes that vx_sparse_decode and vx_block_topk_decode need for this geometry,
  * row bound, k and split count (0 = the planned count); 0 when the arguments are
- * invalid (see vx_last_error).  Deterministic: the same inputs give the same size.
+ * invalid (see vx_last_error).  Deterministic: the same inputs give the same size.  The
+ * layout starts with a fixed-size counter region of the persistent fused step (see
+ * vx_block_topk_decode_persistent: zero-fill a workspace once before its first use there).
  */
 size_t vx_workspace_size(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits);
 

@@ -17,8 +17,9 @@
 // Compute: lane l works on page l / (Hkv*S) of the stage, KV head (l / S) % Hkv and
 // segment l % S of that head's row (DPL = D / S dims, kept as the summed query in
 // registers), so a dot product is DPL FMAs plus a log2(S)-step shuffle; each lane walks
-// its 16-byte chunks in an order rotated by its lane id, which keeps the shared-memory
-// reads free of bank conflicts.  Scores are collected in a per-warp [Hkv][32] buffer and
+// its 16-byte chunks in an order rotated by its place in the page's lane group, which keeps
+// the shared-memory reads free of bank conflicts when a group spans 8 or more lanes and
+// fixes every page's sum order whatever stage slot it lands in.  Scores are collected in a per-warp [Hkv][32] buffer and
 // written as coalesced 128-byte rows.
 #include "vx_internal.h"
 
@@ -82,6 +83,10 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
     const int my_page = lane / lanes_per_page;
     const int my_head = (lane / S) % a.Hkv;
     const int my_seg = lane % S;
+    // chunk rotation of the dot products: fixed by (head, segment), not by the page's slot in
+    // a stage, so a page's sum order never depends on how stages were cut (16-byte reads of
+    // the lanes of one page group hit distinct banks once the group spans 8 lanes)
+    const int rot_lane = (lane % lanes_per_page) % NCH;
 
     extern __shared__ __align__(128) uint8_t smem[];
     int *prefix = reinterpret_cast<int *>(smem);  // B + 1: pages of request b = [prefix[b], prefix[b+1])
@@ -191,8 +196,8 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
 #pragma unroll
                 for (int i = 0; i < 8; ++i) qreg[c][i] += __shfl_xor_sync(FULL, qreg[c][i], off);
         }
-        // rotate: qreg[c] <- chunk (c + lane) % NCH
-        const int rot = lane % NCH;
+        // rotate: qreg[c] <- chunk (c + rot) % NCH, rot = the lane's place in its page group
+        const int rot = rot_lane;
 #pragma unroll
         for (int sh = 1; sh < NCH; sh <<= 1) {
             if (rot & sh) {
@@ -300,7 +305,7 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
             float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
-                const int ch = (c + lane) % NCH;
+                const int ch = (c + rot_lane) % NCH;
                 uint4 v;
                 asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)

@@ -153,17 +153,72 @@ vx_status plan(const vx_geometry *g, int32_t k, int32_t num_splits, Plan *p) {
     return VX_OK;
 }
 
-// workspace layout, every region 256-byte aligned
+// The persistent fused step (GQA geometry, exact top-k, planned splits): its work-item sizes.
+struct FusedPlan {
+    bool ok;               // the geometry and batch fit the fused kernel
+    int32_t spages;        // pages per score item
+    int32_t dtiles;        // tiles per attention item
+    int32_t t_blocks;      // blocks whose warps start on top-k rows
+    int32_t dlag;          // rounds between a request's score items and its attention items
+    int64_t slots;         // partial slots it may use (rows * items per row, at most)
+};
+
+constexpr int FUSED_SPAGES = 16;
+constexpr double FUSED_LAG_BYTES = 120e6;
+constexpr int FUSED_MAX_ITEMS_PER_ROW = 16;
+
+FusedPlan fused_plan(const vx_geometry *g, int32_t max_pages, int32_t k) {
+    FusedPlan f{false, FUSED_SPAGES, 0, 0, 1, 0};
+    const int Hkv = g->num_kv_heads, D = g->head_dim_qk;
+    const int G = g->num_q_heads / Hkv;
+    const int lanes_per_page = Hkv * 2;  // a head row is split over 2 lanes (64 dims at D = 128, 32 at D = 64)
+    if (g->mla_shared_kv || g->head_dim_v != D || (D != 64 && D != 128) || g->batch > vx::FUSED_MAX_B ||
+        Hkv > vx::FUSED_MAX_HKV || lanes_per_page > 32 || 32 % lanes_per_page || G > 16 ||
+        g->page_size % vx::DEC_TILE)
+        return f;
+    int sms = 0;
+    if (sm_count_current(&sms) != 0 || sms < 1) return f;
+    const int64_t tpp = g->page_size / vx::DEC_TILE;
+    const int64_t row_tiles = (int64_t)std::min(k, max_pages) * tpp;
+    const int64_t rows = (int64_t)g->batch * Hkv;
+    // about one attention item per warp, 8..64 tiles, at most 16 items per row
+    int64_t want = std::max<int64_t>(1, rows * row_tiles / ((int64_t)sms * vx::FUSED_WARPS));
+    int64_t dt = 8;
+    while (dt * 2 <= want && dt < 64) dt *= 2;
+    while ((row_tiles + dt - 1) / dt > FUSED_MAX_ITEMS_PER_ROW) dt *= 2;
+    const int64_t per_row = std::max<int64_t>(1, (row_tiles + dt - 1) / dt);
+    // the merging warp keeps per_row x G weights and 2 G totals in its 24 KB region
+    if ((per_row * G + 2 * G) * 4 > 16 * 1024) return f;
+    f.ok = true;
+    f.dtiles = static_cast<int32_t>(dt);
+    f.slots = rows * per_row;
+    // Attention items of request r are handed out about FUSED_LAG_BYTES of streaming after
+    // its score items (about 20 us at HBM speed), so its rows are usually selected by then.
+    const double req_bytes = (double)max_pages * Hkv * D * 2 +
+                             (double)std::min(k, max_pages) * g->page_size * Hkv * 2.0 * D * 2;
+    f.dlag = static_cast<int32_t>(std::min<double>(g->batch, std::max(1.0, std::ceil(FUSED_LAG_BYTES / req_bytes))));
+    // Top-k blocks: enough warps for every row's selection to take about 40 us in total,
+    // at an estimated 3 us + 1 us per 200 pages per row on a warp.
+    const int64_t warp_us = rows * (3 + max_pages / 200);
+    f.t_blocks = static_cast<int32_t>(std::min<int64_t>(std::min(24, sms / 4),
+                                                        std::max<int64_t>(2, warp_us / (40 * vx::FUSED_WARPS))));
+    return f;
+}
+
+// workspace layout, every region 256-byte aligned.  The fused step's sync words come first
+// at a fixed size, so their place never depends on the batch or the page count.
 struct WsLayout {
-    size_t scores, sel, o_part, ml_part, total;
+    size_t sync, scores, sel, o_part, ml_part, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 WsLayout ws_layout(const vx_geometry *g, int32_t max_pages, int32_t k, const Plan &p) {
     WsLayout l;
-    const size_t slots = (size_t)(p.rows + p.chunks);
-    l.o_part = 0;
+    const FusedPlan f = fused_plan(g, max_pages, k);
+    const size_t slots = std::max<size_t>((size_t)(p.rows + p.chunks), f.ok ? (size_t)f.slots : 0);
+    l.sync = 0;
+    l.o_part = up256(vx::FUSED_SYNC_WORDS * sizeof(uint32_t));
     l.ml_part = l.o_part + up256(slots * p.G * g->head_dim_v * sizeof(float));
     l.scores = l.ml_part + up256(slots * p.G * 2 * sizeof(float));
     l.sel = l.scores + up256((size_t)p.rows * max_pages * sizeof(float));
@@ -492,6 +547,79 @@ vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *tabl
     e = vx::launch_topk(topk_args(geo, table, scores, k, seed, sel, err), mode, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
     return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, ws, out, lse, err, s, true);
+}
+
+vx_status vx_block_topk_decode_persistent(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                                          const void *k_cache, const void *v_cache, const void *centroids, int32_t k,
+                                          float sm_scale, void *out, float *lse, float *scores_out, int32_t *sel_out,
+                                          void *ws, size_t ws_bytes, int32_t *err, void *stream) {
+    VX_TRY(check_geo(geo, table));
+    VX_TRY(check_ptr(q, "q"));
+    VX_TRY(check_ptr(k_cache, "k_cache"));
+    VX_TRY(check_ptr(v_cache, "v_cache"));
+    VX_TRY(check_ptr(centroids, "centroids"));
+    VX_TRY(check_ptr(out, "out"));
+    VX_TRY(check_ptr(lse, "lse", true));
+    VX_TRY(check_ptr(scores_out, "scores_out", true));
+    VX_TRY(check_ptr(sel_out, "sel_out", true));
+    VX_TRY(check_k_mode(k, 0));
+    if (geo->mla_shared_kv) return fail(VX_ERR_UNSUPPORTED, "the persistent fused step is for the GQA geometry");
+    if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
+    if (!std::isfinite(sm_scale)) return fail(VX_ERR_INVALID_ARG, "sm_scale must be finite");
+    Plan p;
+    VX_TRY(plan(geo, k, 0, &p));
+    const WsLayout l = ws_layout(geo, table->max_pages, k, p);
+    if (!ws || !al16(ws)) return fail(VX_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+    if (ws_bytes < l.total)
+        return fail(VX_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, l.total);
+    float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<char *>(ws) + l.scores);
+    int32_t *sel = sel_out ? sel_out : reinterpret_cast<int32_t *>(static_cast<char *>(ws) + l.sel);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const FusedPlan f = fused_plan(geo, table->max_pages, k);
+    if (!f.ok)
+        return fail(VX_ERR_UNSUPPORTED, "the persistent fused step needs head_dim_qk == head_dim_v in {64, 128}, "
+                                        "num_kv_heads <= 16, <= 16 query heads per KV head and batch <= %d",
+                    vx::FUSED_MAX_B);
+    {
+        // one persistent launch: score -> exact top-k -> attention -> merge
+        vx::FusedArgs a{};
+        a.page_ptr = table->page_ptr;
+        a.page_indices = table->page_indices;
+        a.seq_lens = table->seq_lens;
+        a.q = static_cast<const __nv_bfloat16 *>(q);
+        a.centroids = static_cast<const __nv_bfloat16 *>(centroids);
+        a.scores = scores;
+        a.sel = sel;
+        a.o_part = reinterpret_cast<float *>(static_cast<char *>(ws) + l.o_part);
+        a.ml_part = reinterpret_cast<float *>(static_cast<char *>(ws) + l.ml_part);
+        a.out = static_cast<__nv_bfloat16 *>(out);
+        a.lse = lse;
+        a.err = err;
+        a.sync = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + l.sync);
+        a.B = geo->batch;
+        a.Hq = geo->num_q_heads;
+        a.Hkv = geo->num_kv_heads;
+        a.G = p.G;
+        a.D = geo->head_dim_qk;
+        a.P = geo->page_size;
+        a.max_pages = table->max_pages;
+        a.k = k;
+        a.tiles_per_page = geo->page_size / vx::DEC_TILE;
+        a.spages = f.spages;
+        a.dtiles = f.dtiles;
+        a.t_blocks = f.t_blocks;
+        a.dlag = f.dlag;
+        a.num_pool_pages = geo->num_pool_pages;
+        const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)geo->head_dim_qk);
+        a.scale_log2 = scale * 1.4426950408889634f;
+        const int64_t page_heads = geo->num_pool_pages * geo->num_kv_heads;
+        CUtensorMap tmK, tmV;
+        VX_TRY(make_cache_map(&tmK, k_cache, geo->head_dim_qk, geo->page_size, page_heads, vx::DEC_TILE));
+        VX_TRY(make_cache_map(&tmV, v_cache, geo->head_dim_v, geo->page_size, page_heads, vx::DEC_TILE));
+        cudaError_t e = vx::launch_fused(a, tmK, tmV, s);
+        if (e != cudaSuccess) return cuda_fail(e, "fused step launch");
+        return VX_OK;
+    }
 }
 
 }  // extern "C"

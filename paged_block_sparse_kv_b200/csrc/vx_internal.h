@@ -85,6 +85,41 @@ struct Resolved {
 };
 
 // ------------------------------------------------------------------ launches
+// Persistent fused step (GQA geometry, exact top-k): one launch scores, selects and attends.
+// Streaming work items (score a span of one request's pages, attend a span of one row's
+// tiles) come in ticket order from one counter; top-k rows, in request order, from a second
+// one, taken first by the warps of the first t_blocks blocks (and by any attention item whose
+// row is not taken yet).  `sync` is a fixed-size region of FUSED_SYNC_WORDS uint32 at the start
+// of the workspace: [ticket, blocks_done, abort, row_ticket, scored[FUSED_MAX_B],
+// row_ready[FUSED_MAX_B * FUSED_MAX_HKV], row_done[FUSED_MAX_B * FUSED_MAX_HKV]].  It is zero
+// before a launch and the last block to finish clears what the launch used.
+constexpr int FUSED_WARPS = 8;
+constexpr int FUSED_MAX_B = 1024;
+constexpr int FUSED_MAX_HKV = 16;
+constexpr int FUSED_SYNC_HDR = 4;
+constexpr size_t FUSED_SYNC_WORDS =
+    FUSED_SYNC_HDR + (size_t)FUSED_MAX_B + 2 * (size_t)FUSED_MAX_B * FUSED_MAX_HKV;
+struct FusedArgs {
+    const int32_t *page_ptr, *page_indices, *seq_lens;
+    const __nv_bfloat16 *q, *centroids;
+    float *scores;            // [B][Hkv][max_pages]
+    int32_t *sel;             // [B][Hkv][k]
+    float *o_part;            // [slots][G][D] unnormalised partial outputs
+    float *ml_part;           // [slots][G][2] (running max in log2 units, running sum)
+    __nv_bfloat16 *out;
+    float *lse;
+    int32_t *err;
+    uint32_t *sync;
+    int32_t B, Hq, Hkv, G, D, P, max_pages, k;
+    int32_t tiles_per_page;   // P / DEC_TILE
+    int32_t spages;           // pages per score item (<= 32)
+    int32_t dtiles;           // tiles per attention item
+    int32_t t_blocks;         // blocks whose warps start on top-k rows
+    int32_t dlag;             // attention items of request r join the ticket order at round r + dlag
+    int64_t num_pool_pages;
+    float scale_log2;         // sm_scale * log2(e)
+};
+
 cudaError_t launch_centroid(const CentroidArgs &a, bool append, cudaStream_t s);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s, bool pdl);
 cudaError_t launch_topk(const TopkArgs &a, int mode, cudaStream_t s, bool pdl);
@@ -93,6 +128,10 @@ cudaError_t launch_decode_gqa(const DecodeArgs &a, const CUtensorMap &tmK, const
 cudaError_t launch_decode_mla(const DecodeArgs &a, const CUtensorMap &tmK, int grid, cudaStream_t s,
                               bool pdl);
 cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl);
+// grid = SM count (one block of FUSED_WARPS warps per SM)
+cudaError_t launch_fused(const FusedArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV, cudaStream_t s);
+// shared memory the fused kernel needs for a batch of B (0 if it cannot run it)
+size_t fused_smem_bytes(int32_t B);
 
 // Host helpers of the C ABI layer (vx_api.cu).
 // Bytes of split partials vx_sparse_decode needs for this problem (validates the geometry).

@@ -22,7 +22,7 @@ VX_DATA_BAD_PAGE_ID, VX_DATA_BAD_SEQ_LEN, VX_DATA_BAD_SELECTION, VX_DATA_TIMEOUT
 
 # every symbol include/vx.h declares
 EXPORTS = ["vx_centroid_update", "vx_score_pages", "vx_topk_pages", "vx_sparse_decode",
-           "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_workspace_size", "vx_planned_splits", "vx_status_string",
+           "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_block_topk_decode_persistent", "vx_workspace_size", "vx_planned_splits", "vx_status_string",
            "vx_last_error", "vx_version"]
 
 
@@ -61,6 +61,7 @@ def lib():
         L.vx_topk_pages.argtypes = [G, T, p, i32, i32, u64, p, p, p]
         L.vx_sparse_decode.argtypes = [G, T, p, p, p, p, i32, f32, i32, p, p, p, sz, p, p]
         L.vx_sparse_decode_noalloc.argtypes = [G, T, p, p, p, p, i32, f32, i32, p, p, p, p]
+        L.vx_block_topk_decode_persistent.argtypes = [G, T, p, p, p, p, i32, f32, p, p, p, p, p, sz, p, p]
         L.vx_block_topk_decode.argtypes = [G, T, p, p, p, p, i32, i32, u64, f32, i32, i32, p, p, p, p, p, sz,
                                            p, p]
         L.vx_workspace_size.argtypes = [G, i32, i32, i32]
@@ -72,7 +73,7 @@ def lib():
         L.vx_last_error.restype = ctypes.c_char_p
         L.vx_version.restype = ctypes.c_char_p
         for name in ("vx_centroid_update", "vx_score_pages", "vx_topk_pages", "vx_sparse_decode",
-                     "vx_sparse_decode_noalloc", "vx_block_topk_decode"):
+                     "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_block_topk_decode_persistent"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -201,3 +202,17 @@ def vx_block_topk_decode(geo: Geometry, table: PageTable, q, k_cache, v_cache, c
                                    score_dims, num_splits, _ptr(out, torch.bfloat16), _ptr(lse, torch.float32),
                                    _ptr(scores_out, torch.float32), _ptr(sel_out, torch.int32), _ptr(ws),
                                    ws.numel() * ws.element_size(), _ptr(err, torch.int32), _stream(stream)))
+
+
+def vx_block_topk_decode_persistent(geo: Geometry, table: PageTable, q, k_cache, v_cache, centroids, k: int, out,
+                                    ws, lse=None, sm_scale=0.0, scores_out=None, sel_out=None, err=None,
+                                    stream=None):
+    """The decode step as one persistent kernel (see include/vx.h).  `ws` (uint8,
+    vx_workspace_size bytes) must be zero-filled once before its first use here (torch.zeros);
+    every call leaves its counters zero again."""
+    _ok(lib().vx_block_topk_decode_persistent(ctypes.byref(geo.c()), ctypes.byref(table.c()), _ptr(q, torch.bfloat16),
+                                              _ptr(k_cache, torch.bfloat16), _ptr(v_cache, torch.bfloat16),
+                                              _ptr(centroids, torch.bfloat16), k, float(sm_scale),
+                                              _ptr(out, torch.bfloat16), _ptr(lse, torch.float32),
+                                              _ptr(scores_out, torch.float32), _ptr(sel_out, torch.int32), _ptr(ws),
+                                              ws.numel() * ws.element_size(), _ptr(err, torch.int32), _stream(stream)))

@@ -62,7 +62,7 @@ def gpu_topk(w, scores, k=None, mode=0, seed=0, err=None):
 def workspace(w, k=None, num_splits=0):
     k = w.spec.k if k is None else k
     n = vx.vx_workspace_size(geometry(w), w.max_pages, k, num_splits)
-    return torch.empty(n, dtype=torch.uint8, device=w.k_cache.device)
+    return torch.zeros(n, dtype=torch.uint8, device=w.k_cache.device)  # the persistent step wants it zero-filled
 
 
 def gpu_decode(w, sel, k=None, num_splits=0, sm_scale=0.0, err=None):
@@ -76,16 +76,30 @@ def gpu_decode(w, sel, k=None, num_splits=0, sm_scale=0.0, err=None):
     return out, lse
 
 
-def gpu_fused(w, cen, k=None, mode=0, seed=0, num_splits=0, err=None, keep=True):
+def gpu_fused(w, cen, k=None, mode=0, seed=0, num_splits=0, err=None, keep=True, ws=None):
     k = w.spec.k if k is None else k
     dev = w.k_cache.device
     out = torch.empty((w.batch, w.spec.num_q_heads, w.spec.head_dim_v), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.batch, w.spec.num_q_heads), dtype=torch.float32, device=dev)
     scores = torch.full((w.batch, w.spec.num_kv_heads, w.max_pages), float("nan"), device=dev) if keep else None
     sel = torch.empty((w.batch, w.spec.num_kv_heads, k), dtype=torch.int32, device=dev) if keep else None
-    ws = workspace(w, k, num_splits)
+    ws = workspace(w, k, num_splits) if ws is None else ws
     vx.vx_block_topk_decode(geometry(w), table(w), w.q, w.k_cache, w.v_cache, cen, k, out, ws, lse=lse, mode=mode,
                             seed=seed, num_splits=num_splits, scores_out=scores, sel_out=sel, err=err)
+    return out, lse, scores, sel
+
+
+def gpu_persistent(w, cen, k=None, err=None, ws=None):
+    """vx_block_topk_decode_persistent; `ws` must have been zero-filled once (workspace() does)."""
+    k = w.spec.k if k is None else k
+    dev = w.k_cache.device
+    out = torch.empty((w.batch, w.spec.num_q_heads, w.spec.head_dim_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.spec.num_q_heads), dtype=torch.float32, device=dev)
+    scores = torch.full((w.batch, w.spec.num_kv_heads, w.max_pages), float("nan"), device=dev)
+    sel = torch.empty((w.batch, w.spec.num_kv_heads, k), dtype=torch.int32, device=dev)
+    ws = workspace(w, k) if ws is None else ws
+    vx.vx_block_topk_decode_persistent(geometry(w), table(w), w.q, w.k_cache, w.v_cache, cen, k, out, ws, lse=lse,
+                                       scores_out=scores, sel_out=sel, err=err)
     return out, lse, scores, sel
 
 

@@ -115,6 +115,22 @@ def test_bad_pointers_and_sizes(L):
                               FAKE, need, None, None) == vx.VX_ERR_INVALID_ARG
 
 
+def test_persistent_step_validation(L):
+    # vx_block_topk_decode_persistent refuses what it cannot run, before any launch
+    tp = ctypes.byref(_table())
+    f0 = ctypes.c_float(0.0)
+    mla = _geo(num_q_heads=16, num_kv_heads=1, head_dim_qk=576, head_dim_v=512, page_size=64, mla_shared_kv=1)
+    assert L.vx_block_topk_decode_persistent(ctypes.byref(mla), tp, FAKE, FAKE, FAKE, FAKE, 4, f0, FAKE, None, None,
+                                             None, FAKE, 1 << 30, None, None) == vx.VX_ERR_UNSUPPORTED
+    gp = ctypes.byref(_geo())
+    assert L.vx_block_topk_decode_persistent(gp, tp, None, FAKE, FAKE, FAKE, 4, f0, FAKE, None, None, None, FAKE,
+                                             1 << 30, None, None) == vx.VX_ERR_INVALID_ARG  # q NULL
+    assert L.vx_block_topk_decode_persistent(gp, tp, FAKE, FAKE, FAKE, FAKE, 0, f0, FAKE, None, None, None, FAKE,
+                                             1 << 30, None, None) == vx.VX_ERR_INVALID_ARG  # k = 0
+    assert L.vx_block_topk_decode_persistent(gp, tp, FAKE, FAKE, None, FAKE, 4, f0, FAKE, None, None, None, FAKE,
+                                             1 << 30, None, None) == vx.VX_ERR_INVALID_ARG  # v_cache NULL
+
+
 def test_workspace_size_is_deterministic_and_monotone(L):
     g = _geo()
     gp = ctypes.byref(g)

@@ -110,7 +110,7 @@ def test_continuous_batching_steps():
     lse = torch.empty((w.batch, spec.num_q_heads), dtype=torch.float32, device=dev)
     scores = torch.empty((w.batch, spec.num_kv_heads, w.max_pages), dtype=torch.float32, device=dev)
     sel = torch.empty((w.batch, spec.num_kv_heads, spec.k), dtype=torch.int32, device=dev)
-    ws = torch.empty(vx.vx_workspace_size(geo, w.max_pages, spec.k), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(vx.vx_workspace_size(geo, w.max_pages, spec.k), dtype=torch.uint8, device=dev)
     ridx = torch.as_tensor(reqs)
     for s in range(spec.steps):
         L = w.seq_lens_at(s)

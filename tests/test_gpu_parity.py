@@ -6,8 +6,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_cases import (check_attention, check_scores, err_word, geometry, gpu_centroids, gpu_decode, gpu_fused,
-                       gpu_scores, gpu_topk, host, recall, table, used_pages, workspace)
+from gpu_cases import (check_attention, check_attention_pair, check_scores, err_word, geometry, gpu_centroids,
+                       gpu_decode, gpu_fused, gpu_persistent, gpu_scores, gpu_topk, host, recall, table, used_pages, workspace)
 from paged_block_sparse_kv_b200 import synth, vx
 
 pytestmark = pytest.mark.gpu
@@ -77,6 +77,14 @@ def test_step_by_step_parity(name):
     assert torch.equal(s_f, s) or np.array_equal(s_f.cpu().numpy(), s.cpu().numpy(), equal_nan=True)
     assert torch.equal(sel_f, sel)
     assert torch.equal(out_f, out) and torch.equal(lse_f, lse)
+    if not w.spec.mla_shared_kv:
+        # persistent fused step: the same scores and selection bits; its own attention split,
+        # so its outputs agree within the attention tolerance
+        out_p, lse_p, s_p, sel_p = gpu_persistent(w, cen, err=err)
+        assert np.array_equal(s_p.cpu().numpy(), s.cpu().numpy(), equal_nan=True)
+        assert torch.equal(sel_p, sel)
+        check_attention(out_p, lse_p, o_orc, l_orc)
+        check_attention_pair(out_p, lse_p, out, lse)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
 
@@ -218,3 +226,28 @@ def test_rope_unaware_score_dims():
     s_orc = oracle.scores(h["q"], h["ptr"], h["idx"], h["L"], 16, w.max_pages, 8, centroids_bf16=synth.bits(cen),
                           score_dims=64)
     check_scores(s, s_orc, h["L"], 16)
+
+
+# vx_block_topk_decode_persistent's counters: a fixed region at the head of the workspace
+# (4 + 1024 + 2 * 1024 * 16 uint32 words)
+FUSED_SYNC_BYTES = (4 + 1024 + 2 * 1024 * 16) * 4
+
+
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "g16_d64_page64", "edges_1tok_fullpage_ragged"])
+def test_persistent_step_repeatable_and_leaves_counters_zero(name):
+    # every call must leave the counters zero, so back-to-back calls on one workspace give the
+    # same bits (the work items are planned from the inputs alone)
+    w = workload(name)
+    cen = gpu_centroids(w)
+    ws = workspace(w)
+    err = err_word()
+    runs = [gpu_persistent(w, cen, ws=ws, err=err) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert int(torch.count_nonzero(ws[:FUSED_SYNC_BYTES]).item()) == 0
+    for r in runs[1:]:
+        for x, y in zip(runs[0], r):
+            if x.dtype == torch.bfloat16:
+                assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+            else:
+                assert np.array_equal(x.cpu().numpy(), y.cpu().numpy(), equal_nan=True)
