@@ -239,22 +239,21 @@ __global__ void __launch_bounds__(FUSED_WARPS * 32, 1)
     const int rot_lane = (lane % lpp) % NCH;
     float qreg[NCH][8];
     auto load_query_sum = [&](int b) {
-        // the pps lanes sharing (head, segment) split the group's heads, issue all loads
-        // first, then combine with an xor butterfly in plain chunk order (same bits on every
-        // copy); a barrel shifter rotates the chunks into the lane's order (c + rot_lane) % NCH
+        // the group's heads summed in head order (fp32), chunk c of qreg holding chunk
+        // (c + rot_lane) % NCH: the standalone scorer's sums, bit for bit
         const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)my_head * a.G) * D + my_seg * DPL;
 #pragma unroll
         for (int c = 0; c < NCH; ++c)
 #pragma unroll
             for (int i = 0; i < 8; ++i) qreg[c][i] = 0.f;
-        for (int g0 = my_page; g0 < a.G; g0 += 2 * pps) {
-            const int g1 = g0 + pps;
+        for (int g = 0; g < a.G; g += 2) {  // two heads' loads in flight, added in head order
             uint4 v0[NCH], v1[NCH];
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
-                v0[c] = __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g0 * D + c * 8));
-                v1[c] = g1 < a.G ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g1 * D + c * 8))
-                                 : make_uint4(0u, 0u, 0u, 0u);
+                const int ch = (c + rot_lane) % NCH;
+                v0[c] = __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g * D + ch * 8));
+                v1[c] = g + 1 < a.G ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)(g + 1) * D + ch * 8))
+                                    : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
@@ -262,30 +261,11 @@ __global__ void __launch_bounds__(FUSED_WARPS * 32, 1)
                 bf16x8_to_f32(v0[c], f);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
-                bf16x8_to_f32(v1[c], f);
+                if (g + 1 < a.G) {
+                    bf16x8_to_f32(v1[c], f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
-            }
-        }
-        for (int off = lpp; off < 32; off <<= 1) {
-#pragma unroll
-            for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) qreg[c][i] += __shfl_xor_sync(FULL, qreg[c][i], off);
-        }
-        const int rot = rot_lane;
-#pragma unroll
-        for (int sh = 1; sh < NCH; sh <<= 1) {
-            if (rot & sh) {
-                float t[NCH][8];
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) t[c][i] = qreg[(c + sh) % NCH][i];
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) qreg[c][i] = t[c][i];
+                    for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
+                }
             }
         }
     };

@@ -14,6 +14,10 @@
 // Data path: each warp owns a ring of SCORE_STAGES stages in shared memory; a stage
 // holds up to PPS consecutive pages of one request, each page row fetched by one 1-D TMA
 // bulk copy (completion counted on the stage's mbarrier).
+// Query: each block first sums the G query heads of every KV head (fp32, heads in order)
+// for the first requests its page range touches (up to SCORE_QCAP, in shared memory, one
+// load round for the whole block); a warp meeting another request sums it itself in the
+// same order.
 // Compute: lane l works on page l / (Hkv*S) of the stage, KV head (l / S) % Hkv and
 // segment l % S of that head's row (DPL = D / S dims, kept as the summed query in
 // registers), so a dot product is DPL FMAs plus a log2(S)-step shuffle; each lane walks
@@ -28,6 +32,7 @@ namespace vx {
 constexpr int SCORE_STAGES = 4;        // stages in flight per warp
 constexpr int SCORE_MAX_BATCH = 4096;  // requests whose prefix fits the block's shared memory
 constexpr int SCORE_MAX_HKV = 16;
+constexpr int SCORE_QCAP = 4;          // requests whose summed query a block keeps in shared memory
 
 // dims per lane for a head dim (the head row is split over D / DPL lanes)
 template <int D>
@@ -92,8 +97,8 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
     int *prefix = reinterpret_cast<int *>(smem);  // B + 1: pages of request b = [prefix[b], prefix[b+1])
     int *pptr = prefix + a.B + 1;                 // B: page_ptr
     const uint32_t head_bytes = ((uint32_t)(2 * a.B + 1) * 4u + 127u) & ~127u;
-    uint8_t *per_warp = smem + head_bytes + (size_t)warp * (SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 +
-                                                            SCORE_STAGES * (8 + sizeof(ScoreMeta)));
+    const size_t per_warp_bytes = SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 + SCORE_STAGES * (8 + sizeof(ScoreMeta));
+    uint8_t *per_warp = smem + head_bytes + (size_t)warp * per_warp_bytes;
     const uint32_t ring0 = smem_u32(per_warp);
     float *tbuf = reinterpret_cast<float *>(per_warp + SCORE_STAGES * stage_bytes);  // [Hkv][32]
     const uint32_t bar0 = smem_u32(per_warp + SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4);
@@ -129,6 +134,48 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
     const int64_t T = prefix[a.B];
     const int64_t W = (int64_t)gridDim.x * SCORE_WARPS;
     const int64_t wid = (int64_t)blockIdx.x * SCORE_WARPS + warp;
+    auto request_of = [&](int64_t p) -> int {  // last b with prefix[b] <= p
+        int lo = 0, hi = a.B - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= p) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    };
+
+    // ---- group-summed queries of the block's first requests, computed once per block: each
+    // thread sums one (request, KV head, 8-dim chunk) over the group's heads in head order
+    float *qs = reinterpret_cast<float *>(smem + head_bytes + (size_t)SCORE_WARPS * per_warp_bytes);  // [qcap][Hkv][D]
+    int qb0 = 0, qn = 0;
+    {
+        const int64_t bp0 = (int64_t)blockIdx.x * SCORE_WARPS * T / W;
+        const int64_t bp1 = ((int64_t)blockIdx.x + 1) * SCORE_WARPS * T / W;
+        if (bp0 < bp1 && a.qcap > 0) {
+            qb0 = request_of(bp0);
+            qn = min(a.qcap, request_of(bp1 - 1) - qb0 + 1);
+        }
+        constexpr int CPR = D / 8;  // 8-dim chunks per head row
+        for (int idx = threadIdx.x; idx < qn * a.Hkv * CPR; idx += blockDim.x) {
+            const int ch = idx % CPR, bh = idx / CPR;
+            const int h = bh % a.Hkv, bq = bh / a.Hkv;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (ch * 8 < a.score_dims) {
+                const __nv_bfloat16 *src = a.q + ((size_t)(qb0 + bq) * a.Hq + (size_t)h * a.G) * D + ch * 8;
+#pragma unroll 4
+                for (int g = 0; g < a.G; ++g) {
+                    float f[8];
+                    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(src + (size_t)g * D)), f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] += f[i];
+                }
+            }
+            float4 *dst = reinterpret_cast<float4 *>(qs + ((size_t)bq * a.Hkv + h) * D + ch * 8);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+        __syncthreads();
+    }
     const int64_t p_begin = wid * T / W, p_end = (wid + 1) * T / W;
     if (p_begin >= p_end) return;
 
@@ -137,12 +184,7 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         rb = -1;
         rj = 0;
         if (p >= p_end) return -1;
-        int lo = 0, hi = a.B - 1;  // last b with prefix[b] <= p
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (prefix[mid] <= p) lo = mid;
-            else hi = mid - 1;
-        }
+        const int lo = request_of(p);
         rb = lo;
         rj = static_cast<int32_t>(p - prefix[lo]);
         const int32_t id = a.page_indices[pptr[lo] + rj];
@@ -153,31 +195,44 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         return id;
     };
 
-    // summed query of request b for this lane's head and segment, in the lane's chunk order.
-    // The pps lanes that share a (head, segment) split the G query heads of the group
-    // between them (lane of page slot d takes heads d, d + pps, ...), issue all their loads
-    // before using any, and combine with an xor butterfly over the page slots (in plain
-    // chunk order, so every copy ends with the same bits and the sum order is fixed); a
-    // barrel shifter then rotates the chunks into the lane's order.
+    // summed query of request b for this lane's head and segment, chunk c of qreg holding
+    // chunk (c + rot_lane) % NCH: from the block's shared copy when the block summed it, else
+    // the same sums (heads in order, fp32) from global memory
     float qreg[NCH][8];
     auto load_query = [&](int b) {
-        const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)my_head * a.G) * D + my_seg * DPL;
-        bool live[NCH];
+        if (b >= qb0 && b < qb0 + qn) {
+            const float *src = qs + ((size_t)(b - qb0) * a.Hkv + my_head) * D + my_seg * DPL;
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            live[c] = my_seg * DPL + c * 8 < a.score_dims;
+            for (int c = 0; c < NCH; ++c) {
+                const float4 *p = reinterpret_cast<const float4 *>(src + ((c + rot_lane) % NCH) * 8);
+                const float4 x = p[0], y = p[1];
+                qreg[c][0] = x.x;
+                qreg[c][1] = x.y;
+                qreg[c][2] = x.z;
+                qreg[c][3] = x.w;
+                qreg[c][4] = y.x;
+                qreg[c][5] = y.y;
+                qreg[c][6] = y.z;
+                qreg[c][7] = y.w;
+            }
+            return;
+        }
+        const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)my_head * a.G) * D + my_seg * DPL;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
 #pragma unroll
             for (int i = 0; i < 8; ++i) qreg[c][i] = 0.f;
-        }
-        for (int g0 = my_page; g0 < a.G; g0 += 2 * pps) {
-            const int g1 = g0 + pps;
+        for (int g = 0; g < a.G; g += 2) {  // two heads' loads in flight, added in head order
             uint4 v0[NCH], v1[NCH];
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
-                v0[c] = live[c] ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g0 * D + c * 8))
-                                : make_uint4(0u, 0u, 0u, 0u);
-                v1[c] = (live[c] && g1 < a.G) ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g1 * D + c * 8))
-                                              : make_uint4(0u, 0u, 0u, 0u);
+                const int ch = (c + rot_lane) % NCH;
+                const bool live = my_seg * DPL + ch * 8 < a.score_dims;
+                v0[c] = live ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)g * D + ch * 8))
+                             : make_uint4(0u, 0u, 0u, 0u);
+                v1[c] = (live && g + 1 < a.G)
+                            ? __ldg(reinterpret_cast<const uint4 *>(qb + (size_t)(g + 1) * D + ch * 8))
+                            : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
@@ -185,31 +240,11 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
                 bf16x8_to_f32(v0[c], f);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
-                bf16x8_to_f32(v1[c], f);
+                if (g + 1 < a.G) {
+                    bf16x8_to_f32(v1[c], f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
-            }
-        }
-        for (int off = lanes_per_page; off < 32; off <<= 1) {
-#pragma unroll
-            for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) qreg[c][i] += __shfl_xor_sync(FULL, qreg[c][i], off);
-        }
-        // rotate: qreg[c] <- chunk (c + rot) % NCH, rot = the lane's place in its page group
-        const int rot = rot_lane;
-#pragma unroll
-        for (int sh = 1; sh < NCH; sh <<= 1) {
-            if (rot & sh) {
-                float t[NCH][8];
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) t[c][i] = qreg[(c + sh) % NCH][i];
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) qreg[c][i] = t[c][i];
+                    for (int i = 0; i < 8; ++i) qreg[c][i] += f[i];
+                }
             }
         }
     };
@@ -360,14 +395,19 @@ static cudaError_t launch_score_d(const ScoreArgs &a, cudaStream_t s, bool pdl) 
     const size_t stage_bytes = ((32 / lpp) * row_bytes + 127) & ~size_t(127);
     const size_t head = ((size_t)(2 * a.B + 1) * 4 + 127) & ~size_t(127);
     const size_t per_warp = SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 + SCORE_STAGES * (8 + sizeof(ScoreMeta));
-    const size_t smem = head + (size_t)SCORE_WARPS * per_warp;
+    size_t smem = head + (size_t)SCORE_WARPS * per_warp;
     // largest need: 4096 requests' prefix (32.9 KB) + 8 warps x 20.6 KB (MLA stages) < 200 KB
     constexpr int SCORE_SMEM_LIMIT = 200 * 1024;
     if (smem > (size_t)SCORE_SMEM_LIMIT) return cudaErrorInvalidValue;
+    // what is left holds the summed queries of up to SCORE_QCAP requests per block
+    ScoreArgs b = a;
+    const size_t q_row = (size_t)a.Hkv * D * sizeof(float);
+    b.qcap = (int32_t)std::min<size_t>(SCORE_QCAP, (SCORE_SMEM_LIMIT - smem) / q_row);
+    smem += (size_t)b.qcap * q_row;
     static std::atomic<unsigned long long> done;
     e = ensure_smem_limit(k_score_pages<D>, SCORE_SMEM_LIMIT, done);
     if (e != cudaSuccess) return e;
-    return launch_k(k_score_pages<D>, dim3(sms), dim3(SCORE_WARPS * 32), smem, s, pdl, a);
+    return launch_k(k_score_pages<D>, dim3(sms), dim3(SCORE_WARPS * 32), smem, s, pdl, b);
 }
 
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s, bool pdl) {

@@ -41,30 +41,30 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t i) {
 
 // Block-wide exclusive scan of one int per thread; also returns the total.  `tmp` holds
 // 32 ints of shared memory.  Contains __syncthreads.
-template <int THREADS>
-__device__ __forceinline__ int block_exclusive_scan(int v, int *tmp, int &total) {
+template <int THREADS, typename V = int>
+__device__ __forceinline__ V block_exclusive_scan(V v, V *tmp, V &total) {
     constexpr int NW = THREADS / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+    V x = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(FULL, x, off);
+        const V y = __shfl_up_sync(FULL, x, off);
         if (lane >= off) x += y;
     }
     if (lane == 31) tmp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = lane < NW ? tmp[lane] : 0;
+        V w = lane < NW ? tmp[lane] : V(0);
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(FULL, w, off);
+            const V y = __shfl_up_sync(FULL, w, off);
             if (lane >= off) w += y;
         }
         if (lane < NW) tmp[lane] = w;  // inclusive over warps
     }
     __syncthreads();
     total = tmp[NW - 1];
-    const int before = (warp > 0 ? tmp[warp - 1] : 0) + x - v;
+    const V before = (warp > 0 ? tmp[warp - 1] : V(0)) + x - v;
     __syncthreads();  // tmp may be reused right after
     return before;
 }
@@ -72,6 +72,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *tmp, int &total)
 struct TopkShared {
     int hist[TOPK_HIST];
     int scan_tmp[32];
+    unsigned long long scan_tmp64[32];
     int bcast[4];
     float fmin[32], fmax[32];
 };
@@ -246,6 +247,32 @@ __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
     };
 
     // -------- ordered compaction
+    if constexpr (!APPROX) {
+        // one counting sweep: keys above the boundary bucket and in it, per thread run; one
+        // scan of both (packed in 64 bits) gives each run its first output slot, since the
+        // bucket's members go out in page order until the slots left are used
+        unsigned long long cnt = 0;
+        for (int j = r0; j < r1; ++j) {
+            const uint32_t mk = key_of(j) & mask;
+            cnt += mk > prefix ? (1ull << 32) : (mk == prefix ? 1ull : 0ull);
+        }
+        unsigned long long tot;
+        const unsigned long long before = block_exclusive_scan<THREADS, unsigned long long>(cnt, sh.scan_tmp64, tot);
+        int eq_rank = static_cast<int>(before & 0xffffffffu);
+        int pos = static_cast<int>(before >> 32) + min(eq_rank, remaining);
+        const int sel_total = static_cast<int>(tot >> 32) + min(static_cast<int>(tot & 0xffffffffu), remaining);
+        for (int j = r0; j < r1; ++j) {
+            const uint32_t mk = key_of(j) & mask;
+            bool take = mk > prefix;
+            if (mk == prefix) take = eq_rank++ < remaining;
+            if (take) {
+                if (pos < a.k) out[pos] = j;
+                ++pos;
+            }
+        }
+        for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;
+        return;
+    }
     // pass 1: rank of each boundary-bucket member among the members in page order
     int eq_local = 0, eq_before_offset_local = 0;
     for (int j = r0; j < r1; ++j) {

@@ -48,6 +48,7 @@ struct ScoreArgs {
     float *scores;
     int32_t *err;
     int32_t B, Hq, Hkv, G, Dqk, P, max_pages, score_dims;
+    int32_t qcap;             // requests whose summed query a block keeps in shared memory
     int64_t num_pool_pages;
 };
 
