@@ -144,6 +144,16 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         return lo;
     };
 
+    const int64_t p_begin = wid * T / W, p_end = (wid + 1) * T / W;
+    // the first batch's page-table reads go out before the block sums the queries, so the
+    // two round trips overlap
+    int32_t pre_raw = -1, pre_b = -1, pre_j = 0;
+    if (p_begin + lane < p_end) {
+        pre_b = request_of(p_begin + lane);
+        pre_j = static_cast<int32_t>(p_begin + lane - prefix[pre_b]);
+        pre_raw = a.page_indices[pptr[pre_b] + pre_j];
+    }
+
     // ---- group-summed queries of the block's first requests, computed once per block: each
     // thread sums one (request, KV head, 8-dim chunk) over the group's heads in head order
     float *qs = reinterpret_cast<float *>(smem + head_bytes + (size_t)SCORE_WARPS * per_warp_bytes);  // [qcap][Hkv][D]
@@ -176,7 +186,6 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         }
         __syncthreads();
     }
-    const int64_t p_begin = wid * T / W, p_end = (wid + 1) * T / W;
     if (p_begin >= p_end) return;
 
     // lane resolves flat page p: request, logical page, physical page (-1: skip)
@@ -265,8 +274,12 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
     };
 
     int64_t batch = p_begin;
-    int32_t my_b, my_j;
-    int32_t my_id = resolve(batch + lane, my_b, my_j);
+    int32_t my_b = pre_b, my_j = pre_j;
+    int32_t my_id = pre_raw;
+    if (my_b >= 0 && (my_id < 0 || my_id >= a.num_pool_pages)) {
+        set_err(a.err, VX_DATA_BAD_PAGE_ID);
+        my_id = -1;
+    }
     uint32_t pending = __ballot_sync(FULL, my_id >= 0);
     uint32_t issued = 0, consumed = 0;
     bool failed = false;
