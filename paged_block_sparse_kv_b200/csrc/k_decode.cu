@@ -279,7 +279,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 // is used, so a row with up to GROUP partials costs one round trip.  The common max comes
 // first (over all partials), then the weighted outputs are summed in partial order.  The
 // launcher picks PER = 1 (more warps, for few rows with many partials) or a wider slice
-// (fewer warps, for many rows with few partials).
+// (fewer warps: for many rows with few partials, or when the narrow shape would not fit in
+// one wave of resident warps).
 template <int DV, int PER, int GROUP>
 __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     pdl_wait();
@@ -402,12 +403,15 @@ static cudaError_t launch_merge_dv(const DecodeArgs &a, cudaStream_t s, bool pdl
     const int64_t wide_items = rows * a.G * (DV / (32 * PW));
     // partials of the row with the most: the chunks it spans
     const int64_t np_max = (a.units_per_row * a.chunks + a.units - 1) / a.units + 1;
-    if (wide_items >= (int64_t)sms * 8 * 4) {  // enough warps for four per SM slot
+    // the narrow shapes keep 24 (16-partial groups) or 16 (32-partial groups) warps resident
+    // per SM; more warps than that would run in several waves
+    const int64_t narrow_items = rows * a.G * (DV / 32);
+    const int64_t narrow_resident = (int64_t)sms * (np_max <= 16 ? 24 : 16);
+    if (wide_items >= (int64_t)sms * 8 * 4 || narrow_items > narrow_resident) {
         const dim3 grid((unsigned)((wide_items + 7) / 8));
         return launch_k(k_merge<DV, PW, 32 / PW>, grid, dim3(256), 0, s, pdl, a);
     }
-    const int64_t items = rows * a.G * (DV / 32);
-    const dim3 grid((unsigned)((items + 7) / 8));
+    const dim3 grid((unsigned)((narrow_items + 7) / 8));
     if (np_max <= 16) return launch_k(k_merge<DV, 1, 16>, grid, dim3(256), 0, s, pdl, a);
     return launch_k(k_merge<DV, 1, 32>, grid, dim3(256), 0, s, pdl, a);
 }
