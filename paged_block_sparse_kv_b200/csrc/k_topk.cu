@@ -246,6 +246,7 @@ __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
         }
     };
 
+    pdl_trigger();  // the decode kernel may land now; only the compaction is left
     // -------- ordered compaction
     if constexpr (!APPROX) {
         // one counting sweep: keys above the boundary bucket and in it, per thread run; one

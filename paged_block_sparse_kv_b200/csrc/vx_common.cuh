@@ -39,12 +39,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 
 // ------------------------------------------------------------------- PDL
 
-// Kernels launched with programmatic dependent launch do not trigger their dependents
-// early: a dependent grid that becomes resident while this one still runs only holds SM
-// resources it cannot use yet (measured slower).  The implicit trigger at block exit still
-// lets the next grid launch as this one drains.
 // Wait until the previous kernel on the stream has finished and its writes are visible.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next grid on the stream launch now (it still waits in pdl_wait for this grid's end
+// and writes).  Only the top-k kernel triggers, late in each block: its dependent (the decode
+// kernel) then lands as top-k blocks leave and runs its prologue meanwhile.  A trigger in the
+// scorer (at its start, or once a warp has issued its last copies) measured slower: top-k
+// blocks fit beside a scorer block and then compete with it; one at the decode kernel's start
+// measured slower and one after its last loads made no difference.  Without a trigger, the
+// next grid launches at block exit.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------------- mbarrier
 
