@@ -73,7 +73,7 @@ def parse():
     ap.add_argument("--copies", type=int, default=0,
                     help="independent input copies to rotate (0: enough for > 3x L2); fewer only for ncu "
                          "captures, which flush the caches before each captured launch themselves")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--persistent", action="store_true",
