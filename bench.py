@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--mode", default="exact", choices=["exact", "approx"])
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--score-dims", type=int, default=0,
+                    help="dims of the key scored against the centroids (0: all; 512 on MLA: rope-unaware)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (small profiling cases only)")
     ap.add_argument("--copies", type=int, default=0,
                     help="independent input copies to rotate (0: enough for > 3x L2); fewer only for ncu "
@@ -223,7 +225,7 @@ def run_vx(args, rank, world, local_rank):
             return
         vx.vx_block_topk_decode(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"], k, c["out"],
                                 c["ws"], lse=c["lse"], mode=mode, seed=0, num_splits=args.splits,
-                                scores_out=c["scores"], sel_out=c["sel"], err=c["err"])
+                                score_dims=args.score_dims, scores_out=c["scores"], sel_out=c["sel"], err=c["err"])
 
     st = []
     if spec.steps == 0:
@@ -475,6 +477,7 @@ def run_vx(args, rank, world, local_rank):
                        "num_kv_heads": spec.num_kv_heads, "head_dim_qk": spec.head_dim_qk,
                        "head_dim_v": spec.head_dim_v, "page_size": spec.page_size, "k_pages": k,
                        "context": list(spec.ctx), "topk_mode": args.mode, "splits": args.splits or "planned",
+                       "score_dims": args.score_dims or spec.head_dim_qk,
                        "entry": "vx_block_topk_decode_persistent" if args.persistent else "vx_block_topk_decode",
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": l2_note.format(n=len(st), mb=mean_bytes * max(1, len(st) - 1) / 1e6)},

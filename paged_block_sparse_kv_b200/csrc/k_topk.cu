@@ -22,7 +22,7 @@
 
 namespace vx {
 
-constexpr int TOPK_SMALL_MAX = 4096;  // rows up to this many pages use 256-thread blocks
+constexpr int TOPK_SMALL_MAX = 6144;  // rows up to this many pages use 256-thread blocks
 constexpr int TOPK_HIST = 1 << APPROX_BITS;
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -120,7 +120,7 @@ __device__ __forceinline__ void sweep_row(const float *row, int n, F &&f) {
 }
 
 template <bool APPROX, int THREADS>
-__global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
+__global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkArgs a) {
     __shared__ TopkShared sh;
     extern __shared__ uint32_t skeys[];  // a.smem_keys entries
     const int b = blockIdx.y, h = blockIdx.x;
@@ -274,51 +274,55 @@ __global__ void __launch_bounds__(THREADS) k_topk(TopkArgs a) {
         for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;
         return;
     }
-    // pass 1: rank of each boundary-bucket member among the members in page order
-    int eq_local = 0, eq_before_offset_local = 0;
+    // approx: members of the boundary code are taken in cyclic page order from `offset`: first
+    // those at or after it (take_hi of them), then those before it (take_lo).  One counting
+    // sweep per run (above / member / member before the offset) and one scan give each run
+    // its first output slot.
+    int gt_l = 0, eq_l = 0, lo_l = 0;
     for (int j = r0; j < r1; ++j) {
-        if ((key_of(j) & mask) == prefix) {
-            ++eq_local;
-            if (j < offset) ++eq_before_offset_local;
+        const uint32_t mk = key_of(j) & mask;
+        if (mk > prefix) ++gt_l;
+        else if (mk == prefix) {
+            ++eq_l;
+            if (j < offset) ++lo_l;
         }
     }
-    int eq_total;
-    const int eq_before = block_exclusive_scan<THREADS>(eq_local, sh.scan_tmp, eq_total);
-    int eq_before_offset = 0;
-    if constexpr (APPROX) {
-        int tmp_total;
-        block_exclusive_scan<THREADS>(eq_before_offset_local, sh.scan_tmp, tmp_total);
-        eq_before_offset = tmp_total;  // members with page index < offset
+    int gt_before, eq_before, lo_before, gt_total, eq_total, lo_total;
+    if (n < (1 << 21)) {  // three 21-bit counts in one 64-bit scan
+        const unsigned long long v = ((unsigned long long)gt_l << 42) | ((unsigned long long)eq_l << 21) | (unsigned long long)lo_l;
+        unsigned long long tot;
+        const unsigned long long bef = block_exclusive_scan<THREADS, unsigned long long>(v, sh.scan_tmp64, tot);
+        constexpr unsigned long long M21 = (1ull << 21) - 1ull;
+        gt_before = (int)(bef >> 42);
+        eq_before = (int)((bef >> 21) & M21);
+        lo_before = (int)(bef & M21);
+        gt_total = (int)(tot >> 42);
+        eq_total = (int)((tot >> 21) & M21);
+        lo_total = (int)(tot & M21);
+    } else {
+        const unsigned long long v = ((unsigned long long)gt_l << 32) | (unsigned long long)eq_l;
+        unsigned long long tot;
+        const unsigned long long bef = block_exclusive_scan<THREADS, unsigned long long>(v, sh.scan_tmp64, tot);
+        gt_before = (int)(bef >> 32);
+        eq_before = (int)(bef & 0xffffffffu);
+        gt_total = (int)(tot >> 32);
+        eq_total = (int)(tot & 0xffffffffu);
+        lo_before = block_exclusive_scan<THREADS>(lo_l, sh.scan_tmp, lo_total);
     }
-    // pass 2: chosen flags, counted per run
-    auto chosen = [&](uint32_t key, int j, int eq_rank) -> bool {
-        const uint32_t mk = key & mask;
-        if (mk > prefix) return true;
-        if (mk != prefix) return false;
-        int r = eq_rank;
-        if constexpr (APPROX) r = (j >= offset) ? eq_rank - eq_before_offset : eq_total - eq_before_offset + eq_rank;
-        return r < remaining;
-    };
-    int sel_local = 0;
+    const int take_hi = min(remaining, eq_total - lo_total);
+    const int take_lo = min(lo_total, remaining - take_hi);
+    int pos = gt_before + min(lo_before, take_lo) + min(eq_before - lo_before, take_hi);
+    const int sel_total = gt_total + take_hi + take_lo;
     {
-        int eq_rank = eq_before;
+        int lo_rank = lo_before, hi_rank = eq_before - lo_before;
         for (int j = r0; j < r1; ++j) {
-            const uint32_t key = key_of(j);
-            if (chosen(key, j, eq_rank)) ++sel_local;
-            if ((key & mask) == prefix) ++eq_rank;
-        }
-    }
-    int sel_total;
-    int pos = block_exclusive_scan<THREADS>(sel_local, sh.scan_tmp, sel_total);
-    {
-        int eq_rank = eq_before;
-        for (int j = r0; j < r1; ++j) {
-            const uint32_t key = key_of(j);
-            if (chosen(key, j, eq_rank)) {
+            const uint32_t mk = key_of(j) & mask;
+            bool take = mk > prefix;
+            if (mk == prefix) take = (j < offset) ? lo_rank++ < take_lo : hi_rank++ < take_hi;
+            if (take) {
                 if (pos < a.k) out[pos] = j;
                 ++pos;
             }
-            if ((key & mask) == prefix) ++eq_rank;
         }
     }
     for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;

@@ -1,12 +1,15 @@
 """GPU parity at the full sizes of the five measured workloads, in the launch
 configuration bench.py times (planned split count, fused call), on sampled requests
 the oracle computes one by one."""
+import math
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from gpu_cases import check_attention, check_scores, err_word, geometry, gpu_centroids, gpu_fused, recall, table
+from gpu_cases import (check_attention, check_scores, err_word, geometry, gpu_centroids, gpu_fused, gpu_scores,
+                       gpu_topk, recall, table)
 from paged_block_sparse_kv_b200 import synth, vx
 
 pytestmark = pytest.mark.gpu
@@ -139,3 +142,42 @@ def test_continuous_batching_steps():
                 cp = init["page_ptr"][i] + pos // P
                 assert np.array_equal(now["k_cache"][now["page_ptr"][i] + pos // P, :, pos % P],
                                       kc[cp, :, pos % P])
+
+
+def test_mla_rope_aware_vs_rope_unaware_selection():
+    # The pages find that routing MLA blocks on the 512 latent dims alone (rope-unaware) loses
+    # accuracy against routing on latent + rope (576 dims).  Without model weights the proxy is
+    # the share of each request's dense attention mass that the selected pages hold; both
+    # selections are exact top-k of their own scores (checked against the oracle bit for bit).
+    name = "mla_576_512_b16"
+    spec = synth.SPECS[name]
+    w = synth.make(spec, 1000 * list(synth.SPECS).index(name), "cuda")
+    cen = gpu_centroids(w)
+    L = w.seq_lens.cpu().numpy()
+    P, k = spec.page_size, spec.k
+    sels = {}
+    for dims in (0, 512):
+        s = gpu_scores(w, cen, score_dims=dims)
+        sel = gpu_topk(w, s)
+        assert np.array_equal(sel.cpu().numpy(), oracle.topk_exact(s.cpu().numpy().astype(np.float64), L, P, k))
+        sels[dims] = sel.cpu().numpy()
+    # dense attention mass per page (plain torch, fp64, on the GPU) for a few requests
+    scale = 1.0 / math.sqrt(spec.head_dim_qk)
+    got = {0: [], 512: []}
+    for b in (0, 5, 10, w.batch - 1):
+        n = (int(L[b]) + P - 1) // P
+        ids = w.page_indices[w.page_ptr[b]:w.page_ptr[b] + n].long()
+        keys = w.k_cache[ids, 0].reshape(n * P, -1)[:int(L[b])].double()           # [L][576]
+        logits = (w.q[b].double() @ keys.T) * scale                                 # [16][L]
+        prob = torch.softmax(logits, dim=-1).mean(dim=0)                            # head-averaged
+        mass = torch.zeros(n * P, dtype=torch.float64, device=prob.device)
+        mass[:int(L[b])] = prob
+        mass = mass.view(n, P).sum(dim=1).cpu().numpy()
+        for dims in (0, 512):
+            chosen = [j for j in sels[dims][b, 0] if j >= 0]
+            got[dims].append(float(mass[chosen].sum()))
+    r = recall(sels[512], sels[0])
+    print(f"\nMLA selection ({name}, k={k}): dense attention mass held, rope-aware {np.mean(got[0]):.4f}, "
+          f"rope-unaware {np.mean(got[512]):.4f}; recall of rope-unaware vs rope-aware {r:.4f}")
+    for dims in (0, 512):
+        assert all(0.0 <= m <= 1.0 + 1e-9 for m in got[dims])
