@@ -173,6 +173,32 @@ def step_bytes(w, sel, seq_lens, k):
     return cen + kv + qo, kv + qo, cen
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+# (weak scaling: every rank runs its own independent batch; the only collectives are a
+# barrier and the max of the timings)
+
+def rank_seed(config, rank):
+    """Seed of rank `rank`'s synthetic workload: independent draws per rank."""
+    from paged_block_sparse_kv_b200 import synth
+    return 1000 * list(synth.SPECS).index(config) + 17 * rank
+
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (every rank must call it, in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(batch_per_rank, ms_per_step, world):
+    """Query tokens per second of the whole job: every rank's batch, at the slowest rank's step time."""
+    return batch_per_rank / (ms_per_step * 1e-3) * world
+
+
 # ------------------------------------------------------------------ our arm
 
 def run_vx(args, rank, world, local_rank):
@@ -198,7 +224,7 @@ def run_vx(args, rank, world, local_rank):
         return vx.Geometry(w.batch, spec.num_q_heads, spec.num_kv_heads, spec.head_dim_qk, spec.head_dim_v,
                            spec.page_size, spec.mla_shared_kv, w.num_pool_pages)
 
-    seed0 = 1000 * (list(synth.SPECS).index(args.config)) + 17 * rank
+    seed0 = rank_seed(args.config, rank)
 
     def buffers(w, geo):
         out = torch.empty((B, spec.num_q_heads, spec.head_dim_v), dtype=torch.bfloat16, device=dev)
@@ -306,11 +332,7 @@ def run_vx(args, rank, world, local_rank):
                 g_rem.replay()
             e1.record(stream)
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         return ms, (g_full, c)
 
     gpu_id = _gpu_id(local_rank)
@@ -326,7 +348,7 @@ def run_vx(args, rank, world, local_rank):
 
     ms_step = ms_total / args.steps
     mean_bytes = sum(p[0] for p in per_copy) / len(per_copy)
-    tok_s = B / (ms_step * 1e-3) * world
+    tok_s = job_throughput(B, ms_step, world)
     peak, peak_kind = peaks()
     step_gbs = mean_bytes / (ms_step * 1e-3) / 1e9
 
@@ -452,12 +474,8 @@ def run_vx(args, rank, world, local_rank):
             g_e.replay()
         ev1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = ev0.elapsed_time(ev1) / (reps * chunk_e)
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / (reps * chunk_e), world, dev)
     del g_e
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
     # the outputs that came back are the call's (a bad copy path would not match)
     for S in sets:
         assert torch.equal(S["h_out"].to(dev), S["d_out"]), "e2e: the D2H copy does not hold the call's outputs"
@@ -491,7 +509,7 @@ def run_vx(args, rank, world, local_rank):
                                                      "csrc/k_decode.cu", args.config, dec_bytes),
                          "bytes_per_launch": int(dec_bytes), "us_per_launch": round(ms_dec_launch * 1e3, 3),
                          "peak_kind": peak_kind},
-            "e2e": {"value": round(B / (ms_e2e * 1e-3) * world, 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "e2e": {"value": round(job_throughput(B, ms_e2e, world), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_e2e, 4),
                     "method": "per step: one H2D of the packed inputs from pinned memory, the public call, one "
                               "D2H of out+lse into pinned memory; copies on their own streams overlapping the "
