@@ -17,9 +17,11 @@
 // partial S tiles are summed through shared memory in a fixed order (so every warp holds
 // the same S), each warp runs the same online softmax (skipping the output rescale when
 // no row maximum moved) and then owns output dims [128w, 128w+128) of P.V.  K tiles
-// (32 x 576 bf16 = 9 TMA boxes of 64 columns x 32 rows, 128-byte swizzle) stream through
-// a MLA_STAGES-deep ring filled by one elected thread; a stage is refilled once every warp
-// has passed the next tile's barrier.
+// (32 x 576 bf16, one TMA copy of 32 whole rows: 288 segments of 128 bytes, segment =
+// token * 9 + 64-column block, 128-byte swizzle by segment index, so the 8 rows of an
+// ldmatrix hit 8 distinct bank groups) stream through a MLA_STAGES-deep ring filled by
+// one elected thread; a stage is refilled once every warp has passed the next tile's
+// barrier.
 #include "vx_internal.h"
 
 namespace vx {
@@ -28,8 +30,7 @@ constexpr int MLA_THREADS = 128;
 constexpr int MLA_STAGES = 2;
 constexpr int MLA_DQK = 576, MLA_DV = 512;
 constexpr int MLA_KB = MLA_DQK / 64;                   // 9 boxes per tile
-constexpr int MLA_BOX = MLA_TILE_TOKENS * 128;         // 4 KB (32 rows x 128 bytes)
-constexpr int MLA_TILE = MLA_KB * MLA_BOX;             // 36 KB
+constexpr int MLA_TILE = MLA_TILE_TOKENS * MLA_DQK * 2;  // 36 KB
 constexpr int MLA_QBOX = 16 * 128;                     // Q: 16 head rows x 128 bytes
 constexpr int MLA_QBYTES = MLA_KB * MLA_QBOX;          // 18 KB
 constexpr int MLA_KSTEPS_PER_WARP = MLA_DQK / 16 / 4;  // 9
@@ -186,8 +187,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
             // their values were consumed before the barrier that released the stage
             mbar_arrive_expect_tx(bar, MLA_TILE);
             const uint32_t dst = sK0 + (uint32_t)st * MLA_TILE;
-#pragma unroll
-            for (int kb = 0; kb < MLA_KB; ++kb) tma_load_3d(dst + kb * MLA_BOX, &tmK, kb * 64, y, z, bar);
+            tma_load_4d(dst, &tmK, 0, 0, y, z, bar);
         }
         __syncwarp();
     };
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
 #pragma unroll
             for (int np = 0; np < MLA_SNT / 2; ++np) {  // pairs of token n-tiles
                 uint32_t kb0, kb1, kb2, kb3;
-                ldsm_x4(sK + box * MLA_BOX + swz128(np * 16 + rr + 8 * (mi >> 1), c0 + (mi & 1)), kb0, kb1, kb2, kb3);
+                ldsm_x4(sK + swz128((np * 16 + rr + 8 * (mi >> 1)) * MLA_KB + box, c0 + (mi & 1)), kb0, kb1, kb2, kb3);
                 mma_bf16_16816(s[2 * np], qa0, qa1, qa2, qa3, kb0, kb1);
                 mma_bf16_16816(s[2 * np + 1], qa0, qa1, qa2, qa3, kb2, kb3);
             }
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(MLA_THREADS, 2)
                 const int ch = warp * 16 + pr * 2;  // 16-byte dim chunk of the first n-tile
                 const int box = ch >> 3, cc = ch & 7;
                 uint32_t v0, v1, v2, v3;
-                ldsm_x4_t(sK + box * MLA_BOX + swz128(ks * 16 + rr + 8 * (mi & 1), cc + (mi >> 1)), v0, v1, v2, v3);
+                ldsm_x4_t(sK + swz128((ks * 16 + rr + 8 * (mi & 1)) * MLA_KB + box, cc + (mi >> 1)), v0, v1, v2, v3);
                 if (tail) {
                     v0 &= mlo;
                     v1 &= mhi;

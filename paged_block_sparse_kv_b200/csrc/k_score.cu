@@ -172,12 +172,20 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (ch * 8 < a.score_dims) {
                 const __nv_bfloat16 *src = a.q + ((size_t)(qb0 + bq) * a.Hq + (size_t)h * a.G) * D + ch * 8;
-#pragma unroll 4
-                for (int g = 0; g < a.G; ++g) {
-                    float f[8];
-                    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(src + (size_t)g * D)), f);
+                for (int g0 = 0; g0 < a.G; g0 += 16) {  // 16 heads' loads in flight, added in head order
+                    uint4 v[16];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] += f[i];
+                    for (int i = 0; i < 16; ++i)
+                        v[i] = g0 + i < a.G ? __ldg(reinterpret_cast<const uint4 *>(src + (size_t)(g0 + i) * D))
+                                            : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (g0 + i >= a.G) break;
+                        float f[8];
+                        bf16x8_to_f32(v[i], f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] += f[e];
+                    }
                 }
             }
             float4 *dst = reinterpret_cast<float4 *>(qs + ((size_t)bq * a.Hkv + h) * D + ch * 8);

@@ -119,10 +119,12 @@ __device__ __forceinline__ void sweep_row(const float *row, int n, F &&f) {
     }
 }
 
+static_assert(TOPK_SMEM_KEYS % 4 == 0, "the key buffer is read in 16-byte vectors");
+
 template <bool APPROX, int THREADS>
 __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkArgs a) {
     __shared__ TopkShared sh;
-    extern __shared__ uint32_t skeys[];  // a.smem_keys entries
+    extern __shared__ __align__(16) uint32_t skeys[];  // a.smem_keys entries, rounded up to 4
     const int b = blockIdx.y, h = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int32_t *out = a.sel + ((size_t)b * a.Hkv + h) * a.k;
@@ -145,8 +147,9 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
     pdl_wait();
     const bool in_smem = n <= a.smem_keys;
 
-    // per-thread contiguous run [r0, r1) used by the ordered compaction
-    const int per = ceil_div(n, THREADS);
+    // per-thread contiguous run [r0, r1) used by the ordered compaction; run starts are
+    // multiples of 4 so a run is read from shared memory as 16-byte vectors
+    const int per = (ceil_div(n, THREADS) + 3) & ~3;
     const int r0 = min(n, tid * per), r1 = min(n, r0 + per);
 
     uint32_t prefix = 0, mask = 0;  // chosen iff (key & mask) > prefix, or == and rank < remaining
@@ -235,8 +238,8 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
         offset = static_cast<int>(splitmix64(a.seed, (uint64_t)b * a.Hkv + h) % (uint64_t)n);
     }
 
-    auto key_of = [&](int j) -> uint32_t {
-        if (in_smem) return skeys[j];
+    // the key of page j computed from its score (rows too long for shared memory)
+    auto key_of_row = [&](int j) -> uint32_t {
         if constexpr (APPROX) {
             if (flat) return 0u;
             const float f = floorf(__fmul_rn(__fsub_rn(row[j], lo), scale));
@@ -245,7 +248,20 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
             return order_key(row[j]);
         }
     };
-
+    // calls fn(j, key of page j) for the pages j of this thread's run, in order
+    auto run_keys = [&](auto &&fn) {
+        if (in_smem) {
+            for (int j4 = r0; j4 < r1; j4 += 4) {
+                const uint4 k4 = *reinterpret_cast<const uint4 *>(skeys + j4);
+                const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (j4 + e < r1) fn(j4 + e, kk[e]);
+            }
+        } else {
+            for (int j = r0; j < r1; ++j) fn(j, key_of_row(j));
+        }
+    };
     pdl_trigger();  // the decode kernel may land now; only the compaction is left
     // -------- ordered compaction
     if constexpr (!APPROX) {
@@ -253,24 +269,24 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
         // scan of both (packed in 64 bits) gives each run its first output slot, since the
         // bucket's members go out in page order until the slots left are used
         unsigned long long cnt = 0;
-        for (int j = r0; j < r1; ++j) {
-            const uint32_t mk = key_of(j) & mask;
+        run_keys([&](int, uint32_t key) {
+            const uint32_t mk = key & mask;
             cnt += mk > prefix ? (1ull << 32) : (mk == prefix ? 1ull : 0ull);
-        }
+        });
         unsigned long long tot;
         const unsigned long long before = block_exclusive_scan<THREADS, unsigned long long>(cnt, sh.scan_tmp64, tot);
         int eq_rank = static_cast<int>(before & 0xffffffffu);
         int pos = static_cast<int>(before >> 32) + min(eq_rank, remaining);
         const int sel_total = static_cast<int>(tot >> 32) + min(static_cast<int>(tot & 0xffffffffu), remaining);
-        for (int j = r0; j < r1; ++j) {
-            const uint32_t mk = key_of(j) & mask;
+        run_keys([&](int j, uint32_t key) {
+            const uint32_t mk = key & mask;
             bool take = mk > prefix;
             if (mk == prefix) take = eq_rank++ < remaining;
             if (take) {
                 if (pos < a.k) out[pos] = j;
                 ++pos;
             }
-        }
+        });
         for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;
         return;
     }
@@ -279,14 +295,14 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
     // sweep per run (above / member / member before the offset) and one scan give each run
     // its first output slot.
     int gt_l = 0, eq_l = 0, lo_l = 0;
-    for (int j = r0; j < r1; ++j) {
-        const uint32_t mk = key_of(j) & mask;
+    run_keys([&](int j, uint32_t key) {
+        const uint32_t mk = key & mask;
         if (mk > prefix) ++gt_l;
         else if (mk == prefix) {
             ++eq_l;
             if (j < offset) ++lo_l;
         }
-    }
+    });
     int gt_before, eq_before, lo_before, gt_total, eq_total, lo_total;
     if (n < (1 << 21)) {  // three 21-bit counts in one 64-bit scan
         const unsigned long long v = ((unsigned long long)gt_l << 42) | ((unsigned long long)eq_l << 21) | (unsigned long long)lo_l;
@@ -315,15 +331,15 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
     const int sel_total = gt_total + take_hi + take_lo;
     {
         int lo_rank = lo_before, hi_rank = eq_before - lo_before;
-        for (int j = r0; j < r1; ++j) {
-            const uint32_t mk = key_of(j) & mask;
+        run_keys([&](int j, uint32_t key) {
+            const uint32_t mk = key & mask;
             bool take = mk > prefix;
             if (mk == prefix) take = (j < offset) ? lo_rank++ < take_lo : hi_rank++ < take_hi;
             if (take) {
                 if (pos < a.k) out[pos] = j;
                 ++pos;
             }
-        }
+        });
     }
     for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;
 }
@@ -331,7 +347,7 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
 template <int THREADS>
 static cudaError_t launch_topk_t(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
     const dim3 grid(a.Hkv, a.B);
-    const size_t smem = sizeof(uint32_t) * (size_t)a.smem_keys;
+    const size_t smem = sizeof(uint32_t) * (size_t)((a.smem_keys + 3) & ~3);  // 16-byte run reads
     auto kern = mode == 0 ? k_topk<false, THREADS> : k_topk<true, THREADS>;
     static std::atomic<unsigned long long> done[2];
     cudaError_t e = ensure_smem_limit(kern, (int)(sizeof(uint32_t) * TOPK_SMEM_KEYS), done[mode]);

@@ -261,6 +261,25 @@ vx_status make_cache_map(CUtensorMap *map, const void *ptr, int dim, int page_si
     return VX_OK;
 }
 
+// Whole token rows in one copy: the row of `dim` bf16 values is viewed as dim / 64 blocks
+// of 64 columns (128 bytes, the 128-byte swizzle span), so a box of (64, dim / 64,
+// box_rows, 1) lands box_rows full rows in shared memory as consecutive 128-byte segments
+// (segment = row * (dim / 64) + block), each swizzled by its segment index.
+vx_status make_cache_map_rows(CUtensorMap *map, const void *ptr, int dim, int page_size, int64_t page_heads,
+                              int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[4] = {64, (cuuint64_t)(dim / 64), (cuuint64_t)page_size, (cuuint64_t)page_heads};
+    cuuint64_t gstride[3] = {128, (cuuint64_t)dim * 2, (cuuint64_t)dim * 2 * page_size};
+    cuuint32_t box[4] = {64, (cuuint32_t)(dim / 64), (cuuint32_t)box_rows, 1};
+    cuuint32_t estride[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return VX_OK;
+}
+
 // ------------------------------------------------------------------ shared launch pieces
 
 vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q, const void *k_cache,
@@ -297,7 +316,7 @@ vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q,
     cudaError_t e;
     if (p.mla) {
         CUtensorMap tmK;
-        VX_TRY(make_cache_map(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::MLA_TILE_TOKENS));
+        VX_TRY(make_cache_map_rows(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::MLA_TILE_TOKENS));
         e = vx::launch_decode_mla(a, tmK, p.grid, s, pdl);
     } else {
         CUtensorMap tmK, tmV;
