@@ -17,8 +17,9 @@
 // live in the pool.
 //
 // Per warp: a ring of DEC_STAGES stages in shared memory, each holding one K tile and
-// one V tile (16 tokens x D bf16 each), filled by TMA tensor loads (128-byte swizzle,
-// 64-column boxes) that complete on a per-stage mbarrier.  Unit metadata (selected
+// one V tile (16 tokens x D bf16 each), each filled by one TMA tensor load (128-byte
+// swizzle; a 4-D view lands the tile as D / 64 consecutive boxes of 16 rows x 64 columns)
+// that completes on a per-stage mbarrier.  Unit metadata (selected
 // page, physical page, valid tokens) is resolved 32 units at a time, one per lane.
 // Per tile: S^T = K Q^T with mma.m16n8k16 (tokens x heads, heads padded to 8 per
 // n-tile), online softmax in base 2, P^T moved into the B-operand layout with
@@ -225,11 +226,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
                 // no proxy fence: this stage's earlier shared-memory reads have completed,
                 // their values were consumed before the __syncwarp that released the stage
                 mbar_arrive_expect_tx(bar, STAGE_BYTES);
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_3d(sK + kb * BOX_BYTES, &tmK, kb * 64, y, z, bar);
-                    tma_load_3d(sK + TILE_BYTES + kb * BOX_BYTES, &tmV, kb * 64, y, z, bar);
-                }
+                tma_load_4d(sK, &tmK, 0, y, 0, z, bar);
+                tma_load_4d(sK + TILE_BYTES, &tmV, 0, y, 0, z, bar);
             }
             __syncwarp();
             ++issued;

@@ -280,6 +280,25 @@ vx_status make_cache_map_rows(CUtensorMap *map, const void *ptr, int dim, int pa
     return VX_OK;
 }
 
+// A tile of box_rows token rows in one copy, laid out as the per-64-column boxes of
+// make_cache_map: the 4-D view (64 columns, rows, dim / 64 column blocks, page-heads) puts
+// the column block outside the rows, so shared memory receives block 0's box_rows x 128
+// bytes, then block 1's, each 128-byte row swizzled by its row index.
+vx_status make_cache_map_blocks(CUtensorMap *map, const void *ptr, int dim, int page_size, int64_t page_heads,
+                                int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[4] = {64, (cuuint64_t)page_size, (cuuint64_t)(dim / 64), (cuuint64_t)page_heads};
+    cuuint64_t gstride[3] = {(cuuint64_t)dim * 2, 128, (cuuint64_t)dim * 2 * page_size};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)(dim / 64), 1};
+    cuuint32_t estride[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return VX_OK;
+}
+
 // ------------------------------------------------------------------ shared launch pieces
 
 vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q, const void *k_cache,
@@ -320,8 +339,8 @@ vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q,
         e = vx::launch_decode_mla(a, tmK, p.grid, s, pdl);
     } else {
         CUtensorMap tmK, tmV;
-        VX_TRY(make_cache_map(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::DEC_TILE));
-        VX_TRY(make_cache_map(&tmV, v_cache, g->head_dim_v, g->page_size, page_heads, vx::DEC_TILE));
+        VX_TRY(make_cache_map_blocks(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::DEC_TILE));
+        VX_TRY(make_cache_map_blocks(&tmV, v_cache, g->head_dim_v, g->page_size, page_heads, vx::DEC_TILE));
         e = vx::launch_decode_gqa(a, tmK, tmV, p.grid, s, pdl);
     }
     if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
