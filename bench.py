@@ -272,7 +272,6 @@ def run_vx(args, rank, world, local_rank):
             tab = vx.PageTable(w.page_ptr, w.page_indices, w.seq_lens, w.max_pages)
             st.append(dict(w=w, geo=geo, tab=tab, cen=rebuild_centroids(w, geo, tab), q=w.q, append=False,
                            seq_lens=w.seq_lens, **buffers(w, geo)))
-        launches_per_step = 4
         l2_note = "inputs rotate over {n} independent copies, {mb:.0f} MB between reuses " + (
             "(> 3x L2)" if (n_copies - 1) * total0 > 3 * L2_BYTES else "(fewer than 3x L2: profiling run only)")
     else:
@@ -289,8 +288,10 @@ def run_vx(args, rank, world, local_rank):
                        v_new=w.step_v_new[s_], seq_lens=lens[s_], **shared)
             ctx["sel"] = torch.empty_like(shared["sel"])
             st.append(ctx)
-        launches_per_step = 5
         l2_note = "{n} consecutive appending decode steps over one {mb:.0f} MB-per-step working set (> L2)"
+    # kernels per step: the centroid append (continuous batching), then the fused call's own
+    # (scores, top-k, attention, merge; the persistent entry is one kernel)
+    launches_per_step = (1 if args.persistent else 4) + (1 if st[0]["append"] else 0)
     for c in st:
         fused(c)
     torch.cuda.synchronize()
