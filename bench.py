@@ -579,9 +579,9 @@ def run_reference(args, rank, world, budget_s=150.0):
     import oracle
     from paged_block_sparse_kv_b200 import synth
     spec = synth.SPECS[args.config]
-    w = synth.make(synth.Spec(**{**spec.__dict__, "steps": 0}), 1000 * list(synth.SPECS).index(args.config),
-                   "cpu", batch=min(spec.batch, 2))
-    h = synth.host_subset(w, list(range(w.batch)))
+    n_req = min(spec.batch, 2)  # requests drawn for the sample (the workload's first two)
+    w = synth.make(synth.Spec(**{**spec.__dict__, "steps": 0}), rank_seed(args.config, 0), "cpu", batch=n_req)
+    h = synth.host_subset(w, list(range(n_req)))
     _, cen16 = oracle.centroids(h["k_cache"], h["page_ptr"], h["page_indices"], h["seq_lens"])
     maxp = int(((h["seq_lens"] + spec.page_size - 1) // spec.page_size).max())
     q = synth.bits(w.q)
@@ -605,9 +605,9 @@ def run_reference(args, rank, world, budget_s=150.0):
     for _ in range(args.steps):
         call(hk)
     dt = time.perf_counter() - t0
-    req_per_step = w.batch * hk / spec.num_kv_heads
+    req_per_step = n_req * hk / spec.num_kv_heads
     value = req_per_step * args.steps / dt
-    sample = (f"{w.batch} of {spec.batch} requests, {hk} of {spec.num_kv_heads} KV heads per step "
+    sample = (f"{n_req} of {spec.batch} requests, {hk} of {spec.num_kv_heads} KV heads per step "
               f"(score + exact top-k + attention, fp64)")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
