@@ -40,11 +40,11 @@ DEFAULT_CONFIG = "qwen3_1p7b_gqa_b32"
 # taken on (sha256 of the file), otherwise the bench reports null.  Summaries: profiles/k_decode_gqa_*.md,
 # profiles/k_decode_mla_*.md.
 DECODE_TRAFFIC = {
-    "csrc/k_decode.cu": {"sha256": "1f17347bfcc8c36b8e9bba4adf0ca066f45a8a3d8c21b0a31fa7a3a2b1b04ed7",
-                         "ratio": (67.244544 + 1.540608) / 67.097856, "workload": "qwen3_1p7b_gqa_b32",
+    "csrc/k_decode.cu": {"sha256": "cef6966877baae394024ef4d58b68199d4fad86380a21263ed1f79e472919f42",
+                         "ratio": (67.243776 + 1.478144) / 67.097856, "workload": "qwen3_1p7b_gqa_b32",
                          "note": "captured at batch 8 (67.1 MB), scaled to the full launch by its bytes"},
-    "csrc/k_decode_mla.cu": {"sha256": "a7960aede43728c07db8e904853a66658d6d8cb6b19778089bb1b328c8156430",
-                             "ratio": (38.134784 + 0.329472) / 38.264896, "workload": "mla_576_512_b16",
+    "csrc/k_decode_mla.cu": {"sha256": "f4bb76c122e394136f340b174b39b6fa507b91f1c215d14781b44231915e6def",
+                             "ratio": (38.131456 + 0.141824) / 38.264896, "workload": "mla_576_512_b16",
                              "note": "captured on the full workload (38.3 MB)"},
 }
 
