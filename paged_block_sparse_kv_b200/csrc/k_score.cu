@@ -97,7 +97,11 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
     int *prefix = reinterpret_cast<int *>(smem);  // B + 1: pages of request b = [prefix[b], prefix[b+1])
     int *pptr = prefix + a.B + 1;                 // B: page_ptr
     const uint32_t head_bytes = ((uint32_t)(2 * a.B + 1) * 4u + 127u) & ~127u;
-    const size_t per_warp_bytes = SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 + SCORE_STAGES * (8 + sizeof(ScoreMeta));
+    // each warp's area starts on a 128-byte boundary: its ring takes bulk copies (16-byte
+    // aligned destinations) and 16-byte shared loads, whatever the stage count
+    const size_t per_warp_bytes =
+        (SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 + SCORE_STAGES * (8 + sizeof(ScoreMeta)) + 127) &
+        ~size_t(127);
     uint8_t *per_warp = smem + head_bytes + (size_t)warp * per_warp_bytes;
     const uint32_t ring0 = smem_u32(per_warp);
     float *tbuf = reinterpret_cast<float *>(per_warp + SCORE_STAGES * stage_bytes);  // [Hkv][32]
@@ -415,7 +419,9 @@ static cudaError_t launch_score_d(const ScoreArgs &a, cudaStream_t s, bool pdl) 
     const size_t row_bytes = (size_t)a.Hkv * D * 2;
     const size_t stage_bytes = ((32 / lpp) * row_bytes + 127) & ~size_t(127);
     const size_t head = ((size_t)(2 * a.B + 1) * 4 + 127) & ~size_t(127);
-    const size_t per_warp = SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 + SCORE_STAGES * (8 + sizeof(ScoreMeta));
+    const size_t per_warp =
+        (SCORE_STAGES * stage_bytes + SCORE_MAX_HKV * 32 * 4 + SCORE_STAGES * (8 + sizeof(ScoreMeta)) + 127) &
+        ~size_t(127);
     size_t smem = head + (size_t)SCORE_WARPS * per_warp;
     // largest need: 4096 requests' prefix (32.9 KB) + 8 warps x 20.6 KB (MLA stages) < 200 KB
     constexpr int SCORE_SMEM_LIMIT = 200 * 1024;
