@@ -24,6 +24,7 @@ def _declare(lib):
     i32, i64, u64, dbl, p = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_double, ctypes.c_void_p
     lib.orc_centroids.argtypes = [p, i32, i32, i32, i32, p, p, p, p, p]
     lib.orc_append.argtypes = [p, p, i32, i32, i32, i32, i32, i32, p, p, p, p, p]
+    lib.orc_prefill_write.argtypes = [p, p, i32, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p]
     lib.orc_scores.argtypes = [p, p, p, i32, i32, i32, i32, i32, i32, p, p, p, i32, p]
     lib.orc_topk_exact.argtypes = [p, i32, i32, i32, p, i32, i32, p]
     lib.orc_topk_approx.argtypes = [p, i32, i32, i32, p, i32, i32, i32, u64, p]
@@ -125,6 +126,23 @@ def append(k_cache, v_cache, page_ptr, page_indices, seq_lens, k_new, v_new, mla
     v_new = None if mla_shared_kv else _c(v_new, np.uint16)
     _load().orc_append(_p(k), _p(v), int(mla_shared_kv), hkv, P, dqk, dv, len(seq_lens), _p(page_ptr),
                        _p(page_indices), _p(seq_lens), _p(k_new), _p(v_new))
+    return k, v
+
+
+def prefill_write(k_cache, v_cache, page_ptr, page_indices, seq_lens, first_pos, k_new, v_new, max_len,
+                  mla_shared_kv=False):
+    """Write positions [first_pos[b], seq_lens[b]) of every request, packed in request order in
+    k_new [N][Hkv][Dqk] / v_new [N][Hkv][Dv], into copies of the caches; returns (k, v)."""
+    k = np.array(_c(k_cache, np.uint16), copy=True)
+    v = None if mla_shared_kv else np.array(_c(v_cache, np.uint16), copy=True)
+    npool, hkv, P, dqk = k.shape
+    dv = dqk if v is None else v.shape[-1]
+    page_ptr, page_indices, seq_lens, first_pos = (_c(page_ptr, np.int32), _c(page_indices, np.int32),
+                                                   _c(seq_lens, np.int32), _c(first_pos, np.int32))
+    k_new = _c(k_new, np.uint16)
+    v_new = None if mla_shared_kv else _c(v_new, np.uint16)
+    _load().orc_prefill_write(_p(k), _p(v), int(mla_shared_kv), hkv, P, dqk, dv, len(seq_lens), int(max_len),
+                              _p(page_ptr), _p(page_indices), _p(seq_lens), _p(first_pos), _p(k_new), _p(v_new))
     return k, v
 
 

@@ -164,6 +164,38 @@ int orc_append(uint16_t *k_cache, uint16_t *v_cache, int32_t mla_shared_kv,
     return 0;
 }
 
+/*
+ * Prefill write (cache stage, paper note section 系统设计 1: the cache is filled as tokens
+ * arrive).  Positions [first_pos[b], seq_lens[b]) of request b arrive packed in request
+ * order: k_new [N][Hkv][Dqk] and v_new [N][Hkv][Dv], request b's first row right after the
+ * rows of the requests before it.  Each row goes to slot pos % P of page
+ * page_indices[page_ptr[b] + pos / P].  A request whose length is not in [1, max_len] or
+ * whose first_pos is outside [0, seq_lens[b]] contributes no rows.  The touched pages'
+ * centroids are then plain page means (orc_centroids over the written cache).
+ */
+int orc_prefill_write(uint16_t *k_cache, uint16_t *v_cache, int32_t mla_shared_kv,
+                      int32_t Hkv, int32_t P, int32_t Dqk, int32_t Dv, int32_t B, int32_t max_len,
+                      const int32_t *page_ptr, const int32_t *page_indices, const int32_t *seq_lens,
+                      const int32_t *first_pos, const uint16_t *k_new, const uint16_t *v_new) {
+    int64_t row = 0; /* packed input row of the next new token */
+    for (int32_t b = 0; b < B; ++b) {
+        int32_t L = seq_lens[b], fp = first_pos[b];
+        if (L < 1 || L > max_len || fp < 0 || fp > L) continue;
+        for (int32_t pos = fp; pos < L; ++pos, ++row) {
+            int64_t page = page_indices[page_ptr[b] + pos / P];
+            int32_t in_page = pos % P;
+            for (int32_t h = 0; h < Hkv; ++h) {
+                for (int32_t d = 0; d < Dqk; ++d)
+                    k_cache[((page * Hkv + h) * P + in_page) * Dqk + d] = k_new[(row * Hkv + h) * Dqk + d];
+                if (!mla_shared_kv)
+                    for (int32_t d = 0; d < Dv; ++d)
+                        v_cache[((page * Hkv + h) * P + in_page) * Dv + d] = v_new[(row * Hkv + h) * Dv + d];
+            }
+        }
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------- step 2: indexer */
 
 /*

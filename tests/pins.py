@@ -522,6 +522,81 @@ def pin_append_running_mean():
         assert np.array_equal(k2[phys, :, pos % 16], k_new[b]) and np.array_equal(v2[phys, :, pos % 16], v_new[b])
 
 
+def pin_prefill_write_golden_by_hand():
+    # 2 requests, page size 4, one KV head, 2 dims.  Request 0: pages [3, 1], 6 tokens, of which
+    # positions 2..5 are new; request 1: page [0], 3 tokens, all new.  New rows, packed in request
+    # order, hold (r + 1, -(r + 1)) for packed row r.  Old slots of the pool hold 100 + page*10 + slot.
+    P, npool = 4, 5
+    k = np.zeros((npool, 1, P, 2), np.float32)
+    for pg in range(npool):
+        for sl in range(P):
+            k[pg, 0, sl] = (100 + pg * 10 + sl, 100 + pg * 10 + sl)
+    v = -k
+    ptr = np.array([0, 2], np.int32)
+    idx = np.array([3, 1, 0], np.int32)
+    L = np.array([6, 3], np.int32)
+    fp = np.array([2, 0], np.int32)
+    rows = np.array([[[r + 1.0, -(r + 1.0)]] for r in range(7)], np.float32)  # [7][1][2]
+    k2, v2 = oracle.prefill_write(_bf16_bits(k), _bf16_bits(v), ptr, idx, L, fp, _bf16_bits(rows),
+                                  _bf16_bits(-rows), max_len=8)
+    K = oracle.widen_bf16(k2)[:, 0]
+    # expected, written out by hand from the page table
+    assert K[3, 0].tolist() == [130.0, 130.0] and K[3, 1].tolist() == [131.0, 131.0]  # old tokens kept
+    assert K[3, 2].tolist() == [1.0, -1.0] and K[3, 3].tolist() == [2.0, -2.0]        # positions 2, 3
+    assert K[1, 0].tolist() == [3.0, -3.0] and K[1, 1].tolist() == [4.0, -4.0]        # positions 4, 5
+    assert K[1, 2].tolist() == [112.0, 112.0] and K[1, 3].tolist() == [113.0, 113.0]  # untouched
+    assert K[0, 0].tolist() == [5.0, -5.0] and K[0, 1].tolist() == [6.0, -6.0] and K[0, 2].tolist() == [7.0, -7.0]
+    assert K[0, 3].tolist() == [103.0, 103.0] and K[2].tolist() == [[120.0 + i] * 2 for i in range(4)]
+    assert np.array_equal(oracle.widen_bf16(v2), -oracle.widen_bf16(k2))
+    c64, _ = oracle.centroids(k2, ptr, idx, L)
+    assert c64[3, 0].tolist() == [(130 + 131 + 1 + 2) / 4, (130 + 131 - 1 - 2) / 4]
+    assert c64[1, 0].tolist() == [3.5, -3.5] and c64[0, 0].tolist() == [6.0, -6.0]
+
+
+def pin_prefill_write_one_token_is_append():
+    # one new token per request (first_pos = seq_len - 1) is the decode append
+    w = _small(seed=18, batch=3, num_q_heads=4, num_kv_heads=2, head_dim_qk=32, page_size=16,
+               ctx=("list", [5, 16, 47]))
+    a = _np(w)
+    rng = np.random.default_rng(18)
+    k_new = _bf16_bits(rng.standard_normal((3, 2, 32)).astype(np.float32))
+    v_new = _bf16_bits(rng.standard_normal((3, 2, 32)).astype(np.float32))
+    ka, va = oracle.append(a["k"], a["v"], a["ptr"], a["idx"], a["L"], k_new, v_new)
+    kp, vp = oracle.prefill_write(a["k"], a["v"], a["ptr"], a["idx"], a["L"], a["L"] - 1, k_new, v_new,
+                                  max_len=16 * 3)
+    assert np.array_equal(ka.view(np.int16), kp.view(np.int16)) and np.array_equal(va.view(np.int16), vp.view(np.int16))
+
+
+def pin_prefill_write_chunks_compose():
+    # writing [f, L) at once equals writing [f, mid) with lengths mid, then [mid, L)
+    w = _small(seed=19, batch=3, num_q_heads=4, num_kv_heads=2, head_dim_qk=32, page_size=16,
+               ctx=("list", [70, 33, 100]))
+    a = _np(w)
+    f = np.array([0, 20, 37], np.int32)
+    mid = np.array([40, 33, 64], np.int32)
+    n_all = int((a["L"] - f).sum())
+    rng = np.random.default_rng(19)
+    k_new = _bf16_bits(rng.standard_normal((n_all, 2, 32)).astype(np.float32))
+    v_new = _bf16_bits(rng.standard_normal((n_all, 2, 32)).astype(np.float32))
+    k1, v1 = oracle.prefill_write(a["k"], a["v"], a["ptr"], a["idx"], a["L"], f, k_new, v_new, max_len=128)
+    starts = np.concatenate([[0], np.cumsum(a["L"] - f)])
+    first = np.concatenate([np.arange(starts[b], starts[b] + mid[b] - f[b]) for b in range(3)])
+    second = np.concatenate([np.arange(starts[b] + mid[b] - f[b], starts[b + 1]) for b in range(3)])
+    k2, v2 = oracle.prefill_write(a["k"], a["v"], a["ptr"], a["idx"], mid, f, k_new[first], v_new[first],
+                                  max_len=128)
+    k2, v2 = oracle.prefill_write(k2, v2, a["ptr"], a["idx"], a["L"], mid, k_new[second], v_new[second],
+                                  max_len=128)
+    assert np.array_equal(k1.view(np.int16), k2.view(np.int16)) and np.array_equal(v1.view(np.int16), v2.view(np.int16))
+    # and nothing outside the written positions changed
+    kw = oracle.widen_bf16(k1)
+    k0 = oracle.widen_bf16(a["k"])
+    for b in range(3):
+        for pos in range(int(a["L"][b])):
+            phys = int(a["idx"][a["ptr"][b] + pos // 16])
+            if pos < f[b]:
+                assert np.array_equal(kw[phys, :, pos % 16], k0[phys, :, pos % 16])
+
+
 def pin_decode_step_is_the_composition():
     w = _small(seed=17, batch=2, num_q_heads=8, num_kv_heads=2, head_dim_qk=64, page_size=16,
                ctx=("list", [300, 129]))

@@ -38,6 +38,11 @@ MUTANTS = [
     ("topk_ascending_scores", "if (x->s > y->s) return -1;\n    if (x->s < y->s) return 1;",
      "if (x->s < y->s) return -1;\n    if (x->s > y->s) return 1;"),
     ("splitmix_constant_typo", "0xbf58476d1ce4e5b9ULL", "0xbf58476d1ce4e5b8ULL"),
+    ("prefill_slot_off_by_one", "int32_t in_page = pos % P;", "int32_t in_page = (pos + 1) % P;"),
+    ("prefill_rows_restart_per_request", "if (L < 1 || L > max_len || fp < 0 || fp > L) continue;",
+     "if (L < 1 || L > max_len || fp < 0 || fp > L) continue;\n        row = 0;"),
+    ("prefill_ignores_row_start", "int64_t page = page_indices[page_ptr[b] + pos / P];",
+     "int64_t page = page_indices[pos / P];"),
     ("approx_emits_boundary_bucket", "if (code[j] > bstar) out[filled++] = j;", "if (code[j] >= bstar) out[filled++] = j;"),
     ("approx_fill_not_rotated", "int32_t j = (o + i) % n;", "int32_t j = i;"),
     ("approx_clamp_off_by_one", "c = f >= (double)(nbins - 1) ? nbins - 1 : (int32_t)f;",
