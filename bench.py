@@ -80,6 +80,9 @@ def parse():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--persistent", action="store_true",
                     help="time vx_block_topk_decode_persistent (one persistent kernel) instead of the chained call")
+    ap.add_argument("--prefill-write", action="store_true",
+                    help="time the prefill write instead (vx_centroid_update with first_pos = 0: every token of the "
+                         "workload's contexts into its page slot, with the page centroids) and print its own line")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time the score, top-k and decode calls separately (CUDA events, graphs)")
     return ap.parse_args()
@@ -619,6 +622,66 @@ def run_reference(args, rank, world, budget_s=150.0):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill_write(args, rank, world, local_rank):
+    """Whole-context prefill write of the workload's requests: read the packed new K/V once,
+    write them into their slots and the page centroids; HBM-bound, reported against the copy peak."""
+    import torch
+
+    from paged_block_sparse_kv_b200 import synth, vx
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    spec = synth.SPECS[args.config]
+    w = synth.make(synth.Spec(**{**spec.__dict__, "steps": 0}), rank_seed(args.config, rank), dev)
+    geo = vx.Geometry(w.batch, spec.num_q_heads, spec.num_kv_heads, spec.head_dim_qk, spec.head_dim_v,
+                      spec.page_size, spec.mla_shared_kv, w.num_pool_pages)
+    tab = vx.PageTable(w.page_ptr, w.page_indices, w.seq_lens, w.max_pages)
+    n_tok = int(w.seq_lens.sum())
+    g = torch.Generator(device=dev).manual_seed(5)
+    k_new = torch.randn((n_tok, spec.num_kv_heads, spec.head_dim_qk), generator=g, device=dev).to(torch.bfloat16)
+    v_new = None if spec.mla_shared_kv else torch.randn((n_tok, spec.num_kv_heads, spec.head_dim_v), generator=g,
+                                                        device=dev).to(torch.bfloat16)
+    cen = torch.zeros((w.num_pool_pages, spec.num_kv_heads, spec.head_dim_qk), dtype=torch.bfloat16, device=dev)
+    fp = torch.zeros(w.batch, dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def call():
+        vx.vx_centroid_update(geo, tab, w.k_cache, cen, v_cache=w.v_cache, k_new=k_new, v_new=v_new, first_pos=fp,
+                              err=err, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(1, min(args.steps, 50))
+    with ClockSampler(_gpu_id(local_rank), not args.no_clocks) as clk:
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(steps):
+                call()  # 2.4+ GB per call at the default workload: nothing stays in L2 between calls
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, f"device error word {int(err.item())}"
+    kv_row = spec.num_kv_heads * (spec.head_dim_qk + (0 if spec.mla_shared_kv else spec.head_dim_v)) * 2
+    pages = int(((w.seq_lens + spec.page_size - 1) // spec.page_size).sum())
+    algo = 2 * n_tok * kv_row + pages * spec.num_kv_heads * spec.head_dim_qk * 2  # read + write, centroids
+    peak, peak_kind = peaks()
+    gbs = algo / (ms * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({"metric": "prefill write (KV slots + page centroids) GB/s", "value": round(gbs * world, 1),
+                          "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": max(3, args.warmup),
+                          "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+                          "dtype": "bf16", "data": "synthetic",
+                          "config": {"workload": args.config, "tokens": n_tok, "pages": pages,
+                                     "bytes_per_call": algo, "entry": "vx_centroid_update (first_pos = 0)"},
+                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                                       "frac": round(gbs / peak, 4), "peak_kind": peak_kind},
+                          "gpu_launches": steps, "clocks": clk.summary()}), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -626,6 +689,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.prefill_write:
+        run_prefill_write(args, rank, world, local_rank)
         return
     run_vx(args, rank, world, local_rank)
 

@@ -101,12 +101,22 @@ typedef struct {
  *   k_new == NULL: rebuild.  Recompute the centroid of every page of every request
  *       holding a position >= first_pos[b] (first_pos NULL: every page).  Use after a
  *       prefill or a bulk load.  v_cache, v_new unused.
- *   k_new != NULL: append one decode token per request.  seq_lens already counts the
- *       new token and its page is installed in the table; the token (k_new [B][Hkv][Dqk],
- *       v_new [B][Hkv][Dv], v_new ignored for MLA) is written into slot
- *       (seq_lens[b]-1) % P of its page and that page's centroid is recomputed from its
- *       keys.  first_pos unused.
- * Writes: centroids (and, when appending, one slot of k_cache / v_cache per request).
+ *   k_new != NULL, first_pos == NULL: append one decode token per request.  seq_lens
+ *       already counts the new token and its page is installed in the table; the token
+ *       (k_new [B][Hkv][Dqk], v_new [B][Hkv][Dv], v_new ignored for MLA) is written into
+ *       slot (seq_lens[b]-1) % P of its page and that page's centroid is recomputed from
+ *       its keys.
+ *   k_new != NULL, first_pos != NULL: prefill write (a prompt or a chunk of one).
+ *       Positions [first_pos[b], seq_lens[b]) of request b arrive packed in request
+ *       order, k_new [N][Hkv][Dqk] and v_new [N][Hkv][Dv] with N = sum over b of
+ *       seq_lens[b] - first_pos[b], request b's rows right after those of requests
+ *       0..b-1; their pages are installed in the table.  One pass writes them into their
+ *       slots and recomputes the centroid of every page they touch (older tokens of the
+ *       first page are read from k_cache).  A request with first_pos[b] == seq_lens[b]
+ *       writes nothing; first_pos[b] outside [0, seq_lens[b]] sets VX_DATA_BAD_SEQ_LEN and
+ *       that request contributes no rows.
+ * Writes: centroids (and, when appending or prefilling, the new tokens' slots of k_cache /
+ * v_cache).
  */
 vx_status vx_centroid_update(const vx_geometry *geo, const vx_page_table *table, void *k_cache,
                              void *v_cache, void *centroids, const void *k_new, const void *v_new,

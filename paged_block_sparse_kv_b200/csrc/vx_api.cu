@@ -469,8 +469,9 @@ vx_status vx_centroid_update(const vx_geometry *geo, const vx_page_table *table,
     VX_TRY(check_geo(geo, table));
     VX_TRY(check_ptr(k_cache, "k_cache"));
     VX_TRY(check_ptr(centroids, "centroids"));
-    const bool append = k_new != nullptr;
-    if (append) {
+    // k_new with first_pos: a prefill chunk per request; k_new alone: one appended token
+    const int mode = k_new ? (first_pos ? vx::CEN_PREFILL : vx::CEN_APPEND) : vx::CEN_REBUILD;
+    if (k_new) {
         VX_TRY(check_ptr(k_new, "k_new"));
         if (!geo->mla_shared_kv) {
             VX_TRY(check_ptr(v_cache, "v_cache"));
@@ -483,7 +484,7 @@ vx_status vx_centroid_update(const vx_geometry *geo, const vx_page_table *table,
     a.page_ptr = table->page_ptr;
     a.page_indices = table->page_indices;
     a.seq_lens = table->seq_lens;
-    a.first_pos = append ? nullptr : first_pos;
+    a.first_pos = mode == vx::CEN_APPEND ? nullptr : first_pos;
     a.k_cache = k_cache;
     a.v_cache = v_cache;
     a.centroids = centroids;
@@ -498,7 +499,7 @@ vx_status vx_centroid_update(const vx_geometry *geo, const vx_page_table *table,
     a.max_pages = table->max_pages;
     a.mla_shared_kv = geo->mla_shared_kv;
     a.num_pool_pages = geo->num_pool_pages;
-    cudaError_t e = vx::launch_centroid(a, append, static_cast<cudaStream_t>(stream));
+    cudaError_t e = vx::launch_centroid(a, mode, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "centroid launch");
     return VX_OK;
 }

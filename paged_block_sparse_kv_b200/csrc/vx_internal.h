@@ -121,7 +121,8 @@ struct FusedArgs {
     float scale_log2;         // sm_scale * log2(e)
 };
 
-cudaError_t launch_centroid(const CentroidArgs &a, bool append, cudaStream_t s);
+constexpr int CEN_REBUILD = 0, CEN_APPEND = 1, CEN_PREFILL = 2;  // vx_centroid_update modes
+cudaError_t launch_centroid(const CentroidArgs &a, int mode, cudaStream_t s);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s, bool pdl);
 cudaError_t launch_topk(const TopkArgs &a, int mode, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_gqa(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,

@@ -157,6 +157,8 @@ def vx_planned_splits(geo: Geometry, max_pages: int, k: int) -> int:
 
 def vx_centroid_update(geo: Geometry, table: PageTable, k_cache, centroids, v_cache=None, k_new=None, v_new=None,
                        first_pos=None, err=None, stream=None):
+    """Rebuild (k_new None), append one token per request (k_new [B][Hkv][Dqk]) or write a
+    prefill chunk (k_new [N][Hkv][Dqk] packed in request order, with first_pos)."""
     _ok(lib().vx_centroid_update(ctypes.byref(geo.c()), ctypes.byref(table.c()), _ptr(k_cache, torch.bfloat16),
                                  _ptr(v_cache, torch.bfloat16), _ptr(centroids, torch.bfloat16),
                                  _ptr(k_new, torch.bfloat16), _ptr(v_new, torch.bfloat16),
