@@ -631,7 +631,8 @@ def run_prefill_write(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     spec = synth.SPECS[args.config]
-    w = synth.make(synth.Spec(**{**spec.__dict__, "steps": 0}), rank_seed(args.config, rank), dev)
+    spec = synth.Spec(**{**spec.__dict__, "steps": 0, **({"batch": args.batch} if args.batch else {})})
+    w = synth.make(spec, rank_seed(args.config, rank), dev)
     geo = vx.Geometry(w.batch, spec.num_q_heads, spec.num_kv_heads, spec.head_dim_qk, spec.head_dim_v,
                       spec.page_size, spec.mla_shared_kv, w.num_pool_pages)
     tab = vx.PageTable(w.page_ptr, w.page_indices, w.seq_lens, w.max_pages)
@@ -675,7 +676,8 @@ def run_prefill_write(args, rank, world, local_rank):
                           "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": max(3, args.warmup),
                           "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
                           "dtype": "bf16", "data": "synthetic",
-                          "config": {"workload": args.config, "tokens": n_tok, "pages": pages,
+                          "config": {"workload": args.config + (f" (batch overridden to {w.batch})" if args.batch else ""),
+                                     "tokens": n_tok, "pages": pages,
                                      "bytes_per_call": algo, "entry": "vx_centroid_update (first_pos = 0)"},
                           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                                        "frac": round(gbs / peak, 4), "peak_kind": peak_kind},
