@@ -146,6 +146,8 @@ vx_status vx_score_pages(const vx_geometry *geo, const vx_page_table *table, con
  *       and max; hi == lo gives 0); one histogram; every page above the boundary code b*
  *       is taken and the slots left are filled from code b* in cyclic page order from
  *       offset SplitMix64(seed) draw number (b * Hkv + h) mod n_b, with no refinement.
+ *   mode 2 (approximate, coarser): the same with 10-bit codes (1024 in place of 4096):
+ *       a cheaper histogram for a larger boundary code.
  * Writes sel [B][Hkv][k]: chosen pages in ascending order, then -1.  k >= 1.
  * Scores must be finite; NaN scores give an unspecified (but in-range) selection.
  */

@@ -121,8 +121,12 @@ __device__ __forceinline__ void sweep_row(const float *row, int n, F &&f) {
 
 static_assert(TOPK_SMEM_KEYS % 4 == 0, "the key buffer is read in 16-byte vectors");
 
-template <bool APPROX, int THREADS>
+// ABITS = 0: exact radix select; otherwise the approximate mode with 2^ABITS remap codes.
+template <int ABITS, int THREADS>
 __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkArgs a) {
+    constexpr bool APPROX = ABITS > 0;
+    constexpr int NCODES = APPROX ? (1 << ABITS) : 2;  // remap codes of the approximate mode
+    static_assert(NCODES <= TOPK_HIST && (!APPROX || NCODES % THREADS == 0), "codes tile the block");
     __shared__ TopkShared sh;
     extern __shared__ __align__(16) uint32_t skeys[];  // a.smem_keys entries, rounded up to 4
     const int b = blockIdx.y, h = blockIdx.x;
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
             sh.fmin[warp] = mn;
             sh.fmax[warp] = mx;
         }
-        for (int i = tid; i < TOPK_HIST; i += THREADS) sh.hist[i] = 0;
+        for (int i = tid; i < NCODES; i += THREADS) sh.hist[i] = 0;
         __syncthreads();
         mn = sh.fmin[0];
         mx = sh.fmax[0];
@@ -218,20 +222,20 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
         }
         lo = mn;
         const float range = __fsub_rn(mx, mn);
-        scale = __fdiv_rn(static_cast<float>(TOPK_HIST), range);
+        scale = __fdiv_rn(static_cast<float>(NCODES), range);
         flat = !(mx > mn) || isinf(scale);
         for (int j = tid; j < n; j += THREADS) {  // each thread rereads only what it staged
             uint32_t code = 0;
             if (!flat) {
                 const float v = in_smem ? __uint_as_float(skeys[j]) : row[j];
                 const float f = floorf(__fmul_rn(__fsub_rn(v, lo), scale));
-                code = f >= float(TOPK_HIST - 1) ? TOPK_HIST - 1 : static_cast<uint32_t>(f);
+                code = f >= float(NCODES - 1) ? NCODES - 1 : static_cast<uint32_t>(f);
             }
             if (in_smem) skeys[j] = code;
             atomicAdd(&sh.hist[code], 1);
         }
         __syncthreads();
-        block_find_bin<THREADS>(sh, TOPK_HIST, keff);
+        block_find_bin<THREADS>(sh, NCODES, keff);
         prefix = static_cast<uint32_t>(sh.bcast[0]);
         mask = 0xffffffffu;
         remaining = keff - sh.bcast[1];
@@ -243,7 +247,7 @@ __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkA
         if constexpr (APPROX) {
             if (flat) return 0u;
             const float f = floorf(__fmul_rn(__fsub_rn(row[j], lo), scale));
-            return f >= float(TOPK_HIST - 1) ? TOPK_HIST - 1 : static_cast<uint32_t>(f);
+            return f >= float(NCODES - 1) ? NCODES - 1 : static_cast<uint32_t>(f);
         } else {
             return order_key(row[j]);
         }
@@ -348,8 +352,9 @@ template <int THREADS>
 static cudaError_t launch_topk_t(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
     const dim3 grid(a.Hkv, a.B);
     const size_t smem = sizeof(uint32_t) * (size_t)((a.smem_keys + 3) & ~3);  // 16-byte run reads
-    auto kern = mode == 0 ? k_topk<false, THREADS> : k_topk<true, THREADS>;
-    static std::atomic<unsigned long long> done[2];
+    auto kern = mode == 0 ? k_topk<0, THREADS>
+                          : (mode == 1 ? k_topk<APPROX_BITS, THREADS> : k_topk<APPROX_BITS_FAST, THREADS>);
+    static std::atomic<unsigned long long> done[3];
     cudaError_t e = ensure_smem_limit(kern, (int)(sizeof(uint32_t) * TOPK_SMEM_KEYS), done[mode]);
     if (e != cudaSuccess) return e;
     return launch_k(kern, grid, dim3(THREADS), smem, s, pdl, a);

@@ -88,6 +88,12 @@ def test_long_context_approx_mode_recall():
     r = recall(sel_a.cpu().numpy(), sel_exact.cpu().numpy())
     print(f"\nrecall@k approx vs exact ({name}, k={spec.k}): {r:.4f}")
     assert r > 0.9
+    # the coarser remap (1024 codes): bit-exact with the oracle's, and its recall
+    _, _, _, sel_c = gpu_fused(w, cen, mode=2, seed=7)
+    assert np.array_equal(sel_c.cpu().numpy(), oracle.topk_approx(s32, L, spec.page_size, spec.k, 7, bits=10))
+    r10 = recall(sel_c.cpu().numpy(), sel_exact.cpu().numpy())
+    print(f"recall@k approx (1024 codes) vs exact ({name}, k={spec.k}): {r10:.4f}")
+    assert r10 > 0.9
     # attention over the approximate selection is still exact attention over those pages
     reqs = [0, w.batch - 1]
     sub = synth.host_subset(w, reqs)

@@ -142,10 +142,12 @@ def test_approx_topk_bit_exact_on_gpu_scores(name):
     h = host(w)
     s = gpu_scores(w, gpu_centroids(w))
     s32 = s.cpu().numpy()
-    for seed in (0, 12345):
-        sel = gpu_topk(w, s, mode=1, seed=seed)
-        sel_orc = oracle.topk_approx(np.nan_to_num(s32, nan=0.0), h["L"], w.spec.page_size, w.spec.k, seed)
-        assert np.array_equal(sel.cpu().numpy(), sel_orc)
+    for mode, bits in ((1, 12), (2, 10)):
+        for seed in (0, 12345):
+            sel = gpu_topk(w, s, mode=mode, seed=seed)
+            sel_orc = oracle.topk_approx(np.nan_to_num(s32, nan=0.0), h["L"], w.spec.page_size, w.spec.k, seed,
+                                         bits=bits)
+            assert np.array_equal(sel.cpu().numpy(), sel_orc)
     exact = oracle.topk_exact(s32.astype(np.float64), h["L"], w.spec.page_size, w.spec.k)
     assert recall(sel.cpu().numpy(), exact) > 0.5
 
