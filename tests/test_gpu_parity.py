@@ -253,3 +253,52 @@ def test_persistent_step_repeatable_and_leaves_counters_zero(name):
                 assert torch.equal(x.view(torch.int16), y.view(torch.int16))
             else:
                 assert np.array_equal(x.cpu().numpy(), y.cpu().numpy(), equal_nan=True)
+
+
+def test_topk_rows_beyond_shared_memory():
+    """Rows longer than the top-k kernel's shared-memory key buffer (12,288 pages) read their keys
+    from global memory in every pass: exact and both approximate modes against the oracle, with
+    heavy ties (scores rounded to a few values)."""
+    P = 16
+    L = np.array([20000 * P, 13000 * P - 5], np.int32)
+    max_pages = 20000
+    geo = vx.Geometry(2, 4, 2, 64, 64, P, 0, 40000)
+    dev = "cuda"
+    rng = np.random.default_rng(21)
+    s = np.round(rng.standard_normal((2, 2, max_pages)) * 4).astype(np.float32)  # ~25 distinct values
+    s[1, 1, :] = rng.standard_normal(max_pages).astype(np.float32)
+    scores = torch.from_numpy(s).to(dev)
+    seq = torch.from_numpy(L).to(dev)
+    dummy = torch.zeros(4, dtype=torch.int32, device=dev)  # the top-k reads only lengths and scores
+    tab = vx.PageTable(dummy, dummy, seq, max_pages)
+    k = 700
+    err = err_word()
+    sel = torch.full((2, 2, k), -7, dtype=torch.int32, device=dev)
+    vx.vx_topk_pages(geo, tab, scores, k, sel, mode=0, err=err)
+    assert np.array_equal(sel.cpu().numpy(), oracle.topk_exact(s.astype(np.float64), L, P, k))
+    for mode, bits in ((1, 12), (2, 10)):
+        vx.vx_topk_pages(geo, tab, scores, k, sel, mode=mode, seed=99, err=err)
+        assert np.array_equal(sel.cpu().numpy(), oracle.topk_approx(s, L, P, k, 99, bits=bits))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+
+
+def test_largest_batch_step():
+    """The whole chained step at the largest batch the library accepts (4,096 requests)."""
+    spec = synth.custom_spec(batch=4096, num_q_heads=4, num_kv_heads=2, head_dim_qk=64, page_size=16,
+                             ctx=("uniform", 1, 120), k=4)
+    w = synth.make(spec, 23, "cuda")
+    h = host(w)
+    err = err_word()
+    cen = gpu_centroids(w, err)
+    out, lse, scores, sel = gpu_fused(w, cen, err=err)
+    s_gpu = scores.cpu().numpy().astype(np.float64)
+    sel_orc = oracle.topk_exact(s_gpu, h["L"], spec.page_size, spec.k)
+    assert np.array_equal(sel.cpu().numpy(), sel_orc)
+    reqs = [0, 1, 2047, 4094, 4095]
+    sub = synth.host_subset(w, reqs)
+    o_orc, l_orc = oracle.attend(synth.bits(w.q[reqs]), sub["k_cache"], sub["v_cache"], sub["page_ptr"],
+                                 sub["page_indices"], sub["seq_lens"], sel=sel[reqs].cpu().numpy())
+    check_attention(out[reqs], lse[reqs], o_orc, l_orc)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
