@@ -59,6 +59,7 @@ struct TopkArgs {
     int32_t *sel;
     int32_t *err;
     int32_t B, Hkv, P, max_pages, k, smem_keys;
+    int32_t warp_max;  // exact rows of at most this many pages go to one warp (0: none)
     uint64_t seed;
 };
 

@@ -302,3 +302,25 @@ def test_largest_batch_step():
     check_attention(out[reqs], lse[reqs], o_orc, l_orc)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
+
+
+def test_topk_many_short_rows_warp_path():
+    """With many rows (>= 4 per SM) exact rows of at most 512 pages are selected by one warp:
+    crafted rows with heavy ties, -0.0 and +0.0, lengths 1..512 pages, against the oracle."""
+    P, B, hkv, max_pages, k = 16, 512, 2, 512, 40
+    rng = np.random.default_rng(31)
+    n = rng.integers(1, max_pages + 1, B)
+    n[:4] = [1, 40, 41, 512]
+    L = (n * P - rng.integers(0, P, B)).clip(1).astype(np.int32)
+    s = np.round(rng.standard_normal((B, hkv, max_pages)) * 3).astype(np.float32)
+    s[::7, 0, ::3] = -0.0
+    s[1::5, 1, :] = rng.standard_normal((len(range(1, B, 5)), max_pages)).astype(np.float32)
+    geo = vx.Geometry(B, 4, hkv, 64, 64, P, 0, 40000)
+    dummy = torch.zeros(4, dtype=torch.int32, device="cuda")
+    tab = vx.PageTable(dummy, dummy, torch.from_numpy(L).cuda(), max_pages)
+    err = err_word()
+    sel = torch.full((B, hkv, k), -7, dtype=torch.int32, device="cuda")
+    vx.vx_topk_pages(geo, tab, torch.from_numpy(s).cuda(), k, sel, mode=0, err=err)
+    assert np.array_equal(sel.cpu().numpy(), oracle.topk_exact(s.astype(np.float64), L, P, k))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
