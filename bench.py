@@ -351,6 +351,26 @@ def run_vx(args, rank, world, local_rank):
             torch.cuda.synchronize()
     clocks = clk.summary()
 
+    # per-step distribution of the appending loop (mean and median over its steps): one graph per
+    # step, replayed back to back with an event between steps (so no overlap across steps)
+    per_step = None
+    if spec.steps:
+        import numpy as np
+        gs = [capture(1, i, fused) for i in range(len(st))]
+        torch.cuda.synchronize()
+        n_ps = 2 * len(st)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ps + 1)]
+        with torch.cuda.stream(stream):
+            for i in range(n_ps):
+                evs[i].record(stream)
+                gs[i % len(st)].replay()
+            evs[n_ps].record(stream)
+        torch.cuda.synchronize()
+        ts = [evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(n_ps)]
+        per_step = {"mean_us": round(float(np.mean(ts)), 2), "p50_us": round(float(np.median(ts)), 2),
+                    "steps": n_ps, "method": "one CUDA graph per step, replayed back to back, events between steps"}
+        del gs
+
     ms_step = ms_total / args.steps
     mean_bytes = sum(p[0] for p in per_copy) / len(per_copy)
     tok_s = job_throughput(B, ms_step, world)
@@ -526,6 +546,8 @@ def run_vx(args, rank, world, local_rank):
         }
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if per_step is not None:
+            line["per_step"] = per_step
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -566,10 +588,28 @@ def cpu_baseline(w, cen, k, seq_lens, q, budget_s=15.0):
     for _ in range(reps):
         oracle.decode_step(*args, **kw)
     dt = time.perf_counter() - t0
-    return {"value": round(len(reqs) * reps / dt, 3), "unit": UNIT, "cores": oracle.num_threads(),
+    cores = oracle.num_threads()
+    # the same call on one core: the first request only, a few seconds
+    args1 = (args[0][:1], h["k_cache"], h["v_cache"], cen_h, h["page_ptr"][:1], h["page_indices"], h["seq_lens"][:1],
+             maxp, k)
+    prev = oracle.set_num_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.decode_step(*args1, **kw)
+        one1 = time.perf_counter() - t0
+        reps1 = max(1, int(budget_s / 3 / max(one1, 1e-6)))
+        t0 = time.perf_counter()
+        for _ in range(reps1):
+            oracle.decode_step(*args1, **kw)
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(prev)
+    return {"value": round(len(reqs) * reps / dt, 3), "unit": UNIT, "cores": cores,
             "kind": "oracle",
             "sample": f"{len(reqs)} of {w.batch} requests x {reps} decode steps (score + exact top-k + "
-                      f"attention, fp64), {dt:.1f} s"}
+                      f"attention, fp64), {dt:.1f} s",
+            "single_thread": {"value": round(reps1 / dt1, 3), "unit": UNIT, "cores": 1,
+                              "sample": f"1 of {w.batch} requests x {reps1} decode steps, {dt1:.1f} s"}}
 
 
 def run_reference(args, rank, world, budget_s=150.0):

@@ -36,6 +36,8 @@ def _declare(lib):
     lib.orc_widen_bf16.argtypes = [p, i64, p]
     lib.orc_narrow_bf16.argtypes = [p, i64, p]
     lib.orc_num_threads.restype = ctypes.c_int
+    lib.orc_set_num_threads.argtypes = [ctypes.c_int]
+    lib.orc_set_num_threads.restype = ctypes.c_int
     return lib
 
 
@@ -79,6 +81,11 @@ def _p(a):
 
 def num_threads() -> int:
     return int(_load().orc_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Threads the following oracle calls use on this host thread; returns the previous count."""
+    return int(_load().orc_set_num_threads(int(n)))
 
 
 def widen_bf16(bits):

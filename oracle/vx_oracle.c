@@ -93,6 +93,19 @@ int orc_num_threads(void) {
 #endif
 }
 
+/* Threads for the following calls on the calling host thread (n < 1: as many as the host has
+ * processors); returns the previous count.  Used to time the baseline on one core. */
+int orc_set_num_threads(int n) {
+#ifdef _OPENMP
+    int prev = omp_get_max_threads();
+    omp_set_num_threads(n > 0 ? n : omp_get_num_procs());
+    return prev;
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
 /* --------------------------------------------------------------- page-table helpers */
 
 static int32_t pages_of(int32_t seq_len, int32_t P) { return (seq_len + P - 1) / P; }
