@@ -10,14 +10,15 @@
 //   exact:  MSB-first radix select with 11/11/10-bit digits: a shared histogram per
 //           digit, the digit holding the k-th largest key found by a block suffix scan,
 //           early exit once the boundary bucket holds exactly the slots left.
-//   approx: fp32 remap of each score to a 12-bit code between the row's min and max,
-//           one 4096-bin histogram, the boundary code b* from a block suffix scan, no
-//           refinement: the slots left are filled from code b* in cyclic page order from
-//           a SplitMix64-drawn offset.
-// Both finish with an ordered compaction (two block-wide exclusive scans over
-// contiguous per-thread runs), so the chosen pages come out in ascending page order and
-// boundary ties go to the lower page index (exact) or to the first pages after the
-// drawn offset (approx).
+//   approx: fp32 remap of each score to a 12-bit (mode 1) or 10-bit (mode 2) code between
+//           the row's min and max, one histogram of the codes, the boundary code b* from a
+//           block suffix scan, no refinement: the slots left are filled from code b* in
+//           cyclic page order from a SplitMix64-drawn offset.
+// Both finish with an ordered compaction over contiguous per-thread runs (one block-wide
+// exclusive scan of packed counts), so the chosen pages come out in ascending page order
+// and boundary ties go to the lower page index (exact) or to the first pages after the
+// drawn offset (approx).  In launches with at least 4 rows per SM, exact rows of at most
+// 512 pages are done by one warp of the block (warp_topk_small).
 #include "vx_internal.h"
 
 namespace vx {
