@@ -99,6 +99,11 @@ def test_bad_pointers_and_sizes(L):
     assert L.vx_centroid_update(gp, tp, None, None, FAKE, None, None, None, None, None) == vx.VX_ERR_INVALID_ARG
     # append needs v_new for GQA
     assert L.vx_centroid_update(gp, tp, FAKE, FAKE, FAKE, FAKE, None, None, None, None) == vx.VX_ERR_INVALID_ARG
+    # prefill write (k_new and first_pos): GQA needs v_cache and v_new; first_pos must be 4-byte aligned
+    assert L.vx_centroid_update(gp, tp, FAKE, None, FAKE, FAKE, FAKE, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_centroid_update(gp, tp, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_centroid_update(gp, tp, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, None, None) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_centroid_update(gp, tp, FAKE, FAKE, FAKE, FAKE + 8, FAKE, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
     # decode: workspace checked before launch (explicit split count: no device query needed)
     assert L.vx_sparse_decode(gp, tp, FAKE, FAKE, FAKE, FAKE, 4, ctypes.c_float(0.0), 8, FAKE, None, None, 0,
                               None, None) == vx.VX_ERR_WORKSPACE
