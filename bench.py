@@ -1,6 +1,6 @@
 """Benchmark: block top-k sparse attention decode over a paged KV cache on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--mode exact|approx|approx1024]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--mode exact|approx|approx1024|approx256]
     python bench.py --impl reference ...     # the fp64 CPU oracle on the host cores
 
 A step is one decode step of one layer: score every page of every request from the
@@ -67,8 +67,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="vx", choices=["vx", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG)
-    ap.add_argument("--mode", default="exact", choices=["exact", "approx", "approx1024"],
-                    help="top-k mode: exact, approximate with 4096 codes, or with 1024 codes")
+    ap.add_argument("--mode", default="exact", choices=["exact", "approx", "approx1024", "approx256"],
+                    help="top-k mode: exact, or approximate with 4096, 1024 or 256 codes")
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--score-dims", type=int, default=0,
                     help="dims of the key scored against the centroids (0: all; 512 on MLA: rope-unaware)")
@@ -220,7 +220,7 @@ def run_vx(args, rank, world, local_rank):
     spec = synth.SPECS[args.config]
     if args.batch:
         spec = synth.Spec(**{**spec.__dict__, "batch": args.batch})
-    mode = {"exact": 0, "approx": 1, "approx1024": 2}[args.mode]
+    mode = {"exact": 0, "approx": 1, "approx1024": 2, "approx256": 3}[args.mode]
     k = spec.k
     B = spec.batch
 

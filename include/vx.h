@@ -148,6 +148,7 @@ vx_status vx_score_pages(const vx_geometry *geo, const vx_page_table *table, con
  *       offset SplitMix64(seed) draw number (b * Hkv + h) mod n_b, with no refinement.
  *   mode 2 (approximate, coarser): the same with 10-bit codes (1024 in place of 4096):
  *       a cheaper histogram for a larger boundary code.
+ *   mode 3 (approximate, coarsest): the same with 8-bit codes (256).
  * Writes sel [B][Hkv][k]: chosen pages in ascending order, then -1.  k >= 1.
  * Scores must be finite; NaN scores give an unspecified (but in-range) selection.
  */

@@ -10,7 +10,7 @@
 //   exact:  MSB-first radix select with 11/11/10-bit digits: a shared histogram per
 //           digit, the digit holding the k-th largest key found by a block suffix scan,
 //           early exit once the boundary bucket holds exactly the slots left.
-//   approx: fp32 remap of each score to a 12-bit (mode 1) or 10-bit (mode 2) code between
+//   approx: fp32 remap of each score to a 12-bit (mode 1), 10-bit (mode 2) or 8-bit (mode 3) code between
 //           the row's min and max, one histogram of the codes, the boundary code b* from a
 //           block suffix scan, no refinement: the slots left are filled from code b* in
 //           cyclic page order from a SplitMix64-drawn offset.
@@ -82,8 +82,11 @@ struct TopkShared {
 // searching from the top: writes (bin, count above it, its count) to sh.bcast.
 template <int THREADS>
 __device__ __forceinline__ void block_find_bin(TopkShared &sh, int bins, int need) {
-    const int per = bins / THREADS;  // bins per thread (bins is a multiple of THREADS)
-    const int base = (THREADS - 1 - (int)threadIdx.x) * per;  // thread 0 owns the top bins
+    // bins per thread: bins / THREADS when bins is a multiple of THREADS, else one for the
+    // first `bins` threads (fewer bins than threads); thread 0 owns the top bins
+    const int tid = static_cast<int>(threadIdx.x);
+    const int per = bins >= THREADS ? bins / THREADS : (tid < bins ? 1 : 0);
+    const int base = bins >= THREADS ? (THREADS - 1 - tid) * per : bins - 1 - tid;
     int own = 0;
     for (int i = 0; i < per; ++i) own += sh.hist[base + i];
     int total;
@@ -247,7 +250,8 @@ template <int ABITS, int THREADS>
 __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkArgs a) {
     constexpr bool APPROX = ABITS > 0;
     constexpr int NCODES = APPROX ? (1 << ABITS) : 2;  // remap codes of the approximate mode
-    static_assert(NCODES <= TOPK_HIST && (!APPROX || NCODES % THREADS == 0), "codes tile the block");
+    static_assert(NCODES <= TOPK_HIST && (!APPROX || NCODES % THREADS == 0 || NCODES < THREADS),
+                  "codes tile the block");
     __shared__ TopkShared sh;
     extern __shared__ __align__(16) uint32_t skeys[];  // a.smem_keys entries, rounded up to 4
     const int b = blockIdx.y, h = blockIdx.x;
@@ -479,9 +483,11 @@ template <int THREADS>
 static cudaError_t launch_topk_t(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
     const dim3 grid(a.Hkv, a.B);
     const size_t smem = sizeof(uint32_t) * (size_t)((a.smem_keys + 3) & ~3);  // 16-byte run reads
-    auto kern = mode == 0 ? k_topk<0, THREADS>
-                          : (mode == 1 ? k_topk<APPROX_BITS, THREADS> : k_topk<APPROX_BITS_FAST, THREADS>);
-    static std::atomic<unsigned long long> done[3];
+    auto kern = mode == 0   ? k_topk<0, THREADS>
+                : mode == 1 ? k_topk<APPROX_BITS, THREADS>
+                : mode == 2 ? k_topk<APPROX_BITS_FAST, THREADS>
+                            : k_topk<APPROX_BITS_COARSE, THREADS>;
+    static std::atomic<unsigned long long> done[4];
     cudaError_t e = ensure_smem_limit(kern, (int)(sizeof(uint32_t) * TOPK_SMEM_KEYS), done[mode]);
     if (e != cudaSuccess) return e;
     return launch_k(kern, grid, dim3(THREADS), smem, s, pdl, a);

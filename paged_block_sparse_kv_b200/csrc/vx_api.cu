@@ -396,8 +396,9 @@ vx_status check_score_dims(const vx_geometry *g, int32_t score_dims) {
 
 vx_status check_k_mode(int32_t k, int32_t mode) {
     if (k < 1) return fail(VX_ERR_INVALID_ARG, "k %d < 1", k);
-    if (mode < 0 || mode > 2)
-        return fail(VX_ERR_INVALID_ARG, "mode %d must be 0 (exact), 1 (approximate, 4096 codes) or 2 (1024 codes)", mode);
+    if (mode < 0 || mode > 3)
+        return fail(VX_ERR_INVALID_ARG,
+                    "mode %d must be 0 (exact), 1 (approximate, 4096 codes), 2 (1024 codes) or 3 (256 codes)", mode);
     return VX_OK;
 }
 

@@ -22,6 +22,7 @@ constexpr int TOPK_THREADS = 1024;       // top-k: one block per (request, KV he
 constexpr int TOPK_SMEM_KEYS = 12288;    // rows up to this many pages keep their keys in smem
 constexpr int APPROX_BITS = 12;          // approximate top-k remap width
 constexpr int APPROX_BITS_FAST = 10;     // approximate top-k, mode 2: 1024 codes
+constexpr int APPROX_BITS_COARSE = 8;    // approximate top-k, mode 3: 256 codes
 constexpr int DEC_WARPS = 8;             // GQA decode: worker warps per block
 constexpr int DEC_STAGES = 3;            // GQA decode: 16-token tiles in flight per warp
 constexpr int DEC_TILE = 16;             // GQA decode: tokens per tile (one mma M or K step)

@@ -95,7 +95,7 @@ def test_bad_pointers_and_sizes(L):
     bad_table = _table(max_pages=0)
     assert L.vx_score_pages(gp, ctypes.byref(bad_table), FAKE, FAKE, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
     assert L.vx_topk_pages(gp, tp, FAKE, 0, 0, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # k = 0
-    assert L.vx_topk_pages(gp, tp, FAKE, 4, 3, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # mode 3
+    assert L.vx_topk_pages(gp, tp, FAKE, 4, 4, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG  # mode 4
     assert L.vx_centroid_update(gp, tp, None, None, FAKE, None, None, None, None, None) == vx.VX_ERR_INVALID_ARG
     # append needs v_new for GQA
     assert L.vx_centroid_update(gp, tp, FAKE, FAKE, FAKE, FAKE, None, None, None, None) == vx.VX_ERR_INVALID_ARG

@@ -94,6 +94,11 @@ def test_long_context_approx_mode_recall():
     r10 = recall(sel_c.cpu().numpy(), sel_exact.cpu().numpy())
     print(f"recall@k approx (1024 codes) vs exact ({name}, k={spec.k}): {r10:.4f}")
     assert r10 > 0.9
+    _, _, _, sel_8 = gpu_fused(w, cen, mode=3, seed=7)
+    assert np.array_equal(sel_8.cpu().numpy(), oracle.topk_approx(s32, L, spec.page_size, spec.k, 7, bits=8))
+    r8 = recall(sel_8.cpu().numpy(), sel_exact.cpu().numpy())
+    print(f"recall@k approx (256 codes) vs exact ({name}, k={spec.k}): {r8:.4f}")
+    assert r8 > 0.8
     # attention over the approximate selection is still exact attention over those pages
     reqs = [0, w.batch - 1]
     sub = synth.host_subset(w, reqs)

@@ -142,7 +142,7 @@ def test_approx_topk_bit_exact_on_gpu_scores(name):
     h = host(w)
     s = gpu_scores(w, gpu_centroids(w))
     s32 = s.cpu().numpy()
-    for mode, bits in ((1, 12), (2, 10)):
+    for mode, bits in ((1, 12), (2, 10), (3, 8)):
         for seed in (0, 12345):
             sel = gpu_topk(w, s, mode=mode, seed=seed)
             sel_orc = oracle.topk_approx(np.nan_to_num(s32, nan=0.0), h["L"], w.spec.page_size, w.spec.k, seed,
@@ -276,7 +276,7 @@ def test_topk_rows_beyond_shared_memory():
     sel = torch.full((2, 2, k), -7, dtype=torch.int32, device=dev)
     vx.vx_topk_pages(geo, tab, scores, k, sel, mode=0, err=err)
     assert np.array_equal(sel.cpu().numpy(), oracle.topk_exact(s.astype(np.float64), L, P, k))
-    for mode, bits in ((1, 12), (2, 10)):
+    for mode, bits in ((1, 12), (2, 10), (3, 8)):
         vx.vx_topk_pages(geo, tab, scores, k, sel, mode=mode, seed=99, err=err)
         assert np.array_equal(sel.cpu().numpy(), oracle.topk_approx(s, L, P, k, 99, bits=bits))
     torch.cuda.synchronize()
