@@ -30,6 +30,8 @@ CASES = {
                                       page_size=64, mla_shared_kv=True, ctx=("list", [700, 2000, 64]), k=6), 17),
     "mla_5heads_ragged": (synth.custom_spec(batch=2, num_q_heads=5, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
                                             page_size=64, mla_shared_kv=True, ctx=("list", [1, 4000]), k=9), 18),
+    "mla_page32": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
+                                     page_size=32, mla_shared_kv=True, ctx=("list", [33, 900, 32]), k=7), 19),
 }
 
 
