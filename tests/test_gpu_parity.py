@@ -326,3 +326,24 @@ def test_topk_many_short_rows_warp_path():
     assert np.array_equal(sel.cpu().numpy(), oracle.topk_exact(s.astype(np.float64), L, P, k))
     torch.cuda.synchronize()
     assert int(err.item()) == 0
+
+
+@pytest.mark.parametrize("name", ["g1_many_rows", "mla_16heads"])
+def test_empty_selection_rows(name):
+    """Rows whose selection is entirely empty (all -1) attend to nothing: out = 0, lse = -inf, as
+    the oracle gives; the other rows are unaffected."""
+    w = workload(name)
+    h = host(w)
+    sel = gpu_topk(w, gpu_scores(w, gpu_centroids(w)))
+    sel[0] = -1            # every KV head of request 0
+    sel[1, 0] = -1         # the first KV head of request 1
+    err = err_word()
+    out, lse = gpu_decode(w, sel, err=err)
+    o_orc, l_orc = oracle.attend(h["q"], h["k"], h["v"], h["ptr"], h["idx"], h["L"], sel=sel.cpu().numpy(),
+                                 **attend_kw(w))
+    G = w.spec.num_q_heads // w.spec.num_kv_heads
+    assert torch.equal(out[0], torch.zeros_like(out[0])) and torch.isneginf(lse[0]).all()
+    assert torch.equal(out[1, :G], torch.zeros_like(out[1, :G])) and torch.isneginf(lse[1, :G]).all()
+    check_attention(out, lse, o_orc, l_orc)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
