@@ -668,9 +668,14 @@ def run_prefill_write(args, rank, world, local_rank):
     write them into their slots and the page centroids; HBM-bound, reported against the copy peak."""
     import torch
 
+    import torch.distributed as dist
+
     from paged_block_sparse_kv_b200 import synth, vx
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     spec = synth.SPECS[args.config]
     spec = synth.Spec(**{**spec.__dict__, "steps": 0, **({"batch": args.batch} if args.batch else {})})
     w = synth.make(spec, rank_seed(args.config, rank), dev)
@@ -723,6 +728,9 @@ def run_prefill_write(args, rank, world, local_rank):
                           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                                        "frac": round(gbs / peak, 4), "peak_kind": peak_kind},
                           "gpu_launches": steps, "clocks": clk.summary()}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def main():
