@@ -37,8 +37,7 @@ DEFAULT_CONFIG = "qwen3_1p7b_gqa_b32"
 
 # DRAM traffic of the dominant kernel from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # as a multiple of the algorithmic bytes of the captured launch; valid only for the kernel source it was
-# taken on (sha256 of the file), otherwise the bench reports null.  Summaries: profiles/k_decode_gqa_*.md,
-# profiles/k_decode_mla_*.md.
+# taken on (sha256 of the file), otherwise the bench reports null.
 DECODE_TRAFFIC = {
     "csrc/k_decode.cu": {"sha256": "cef6966877baae394024ef4d58b68199d4fad86380a21263ed1f79e472919f42",
                          "ratio": (67.243776 + 1.478144) / 67.097856, "workload": "qwen3_1p7b_gqa_b32",
@@ -62,7 +61,8 @@ def measured_traffic(kernel_file, workload, algorithmic_bytes):
 
 def parse():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs of the job; more than 1 needs one process per GPU (torchrun sets WORLD_SIZE)")
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="vx", choices=["vx", "reference"])
@@ -715,10 +715,17 @@ def run_prefill_write(args, rank, world, local_rank):
     kv_row = spec.num_kv_heads * (spec.head_dim_qk + (0 if spec.mla_shared_kv else spec.head_dim_v)) * 2
     pages = int(((w.seq_lens + spec.page_size - 1) // spec.page_size).sum())
     algo = 2 * n_tok * kv_row + pages * spec.num_kv_heads * spec.head_dim_qk * 2  # read + write, centroids
+    # the ranks draw their own contexts, so the job's bytes are the sum over ranks
+    algo_job = algo
+    if world > 1:
+        t = torch.tensor([float(algo)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        algo_job = float(t.item())
     peak, peak_kind = peaks()
     gbs = algo / (ms * 1e-3) / 1e9
     if rank == 0:
-        print(json.dumps({"metric": "prefill write (KV slots + page centroids) GB/s", "value": round(gbs * world, 1),
+        print(json.dumps({"metric": "prefill write (KV slots + page centroids) GB/s",
+                          "value": round(algo_job / (ms * 1e-3) / 1e9, 1),
                           "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": max(3, args.warmup),
                           "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
                           "dtype": "bf16", "data": "synthetic",
@@ -733,11 +740,19 @@ def run_prefill_write(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+def check_world(gpus, world):
+    """--gpus must match the processes launched: one per GPU, WORLD_SIZE set by torchrun."""
+    if gpus != world:
+        raise SystemExit(f"bench.py: --gpus {gpus} but {world} process(es) launched; for N > 1 GPUs launch "
+                         f"one process per GPU with torchrun --nproc-per-node N")
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    check_world(args.gpus, world)
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

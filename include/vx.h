@@ -19,9 +19,11 @@
  *
  * Ownership: the caller allocates and owns every buffer and keeps it alive until the
  * stream has passed the call.  The library allocates no device memory and keeps no
- * device state; calls are asynchronous and stream-ordered and never synchronise the
- * host.  Calls on different streams may run concurrently when they write disjoint
- * buffers (outputs, workspace, err).
+ * device state, with one exception: the fixed scratch array of vx_sparse_decode_noalloc
+ * (one per GPU, held until the process exits, shared by every call of that function).
+ * Calls are asynchronous and stream-ordered and never synchronise the host.  Calls on
+ * different streams may run concurrently when they write disjoint buffers (outputs,
+ * workspace, err).
  *
  * Layouts (row-major, element types in brackets):
  *   k_cache    [num_pool_pages][num_kv_heads][page_size][head_dim_qk]  (bf16)
@@ -224,16 +226,24 @@ vx_status vx_block_topk_decode_persistent(const vx_geometry *geo, const vx_page_
  * no workspace, or a caller that must avoid the device synchronisation cudaMalloc and
  * cudaFree can cause.
  * What it does: exactly vx_sparse_decode (same arguments minus ws / ws_bytes, same
- * results), with the split partials kept in one array of VX_NOALLOC_SCRATCH_BYTES that
- * the library holds in device memory, once per GPU, until the process exits.  It
- * allocates nothing and calls no allocating routine.
- *   - Limit: a problem whose split partials need more than VX_NOALLOC_SCRATCH_BYTES
- *     ((rows + splits) * G * (head_dim_v + 2) * 4 bytes, rows = batch * num_kv_heads)
- *     is rejected with VX_ERR_WORKSPACE and a message; pass fewer splits or use
- *     vx_sparse_decode with your own workspace.
- *   - Set-up: the first call on each device looks the array's device address up
- *     (cudaGetSymbolAddress, with that device current).  Make that first call on a
- *     device before any stream capture.
+ * kernels, same split plan, so bit-identical results for the same num_splits), with the
+ * split partials kept in one array of VX_NOALLOC_SCRATCH_BYTES that the library holds in
+ * device memory, once per GPU, until the process exits.  It calls no cudaMalloc, cudaFree
+ * or other allocating routine.
+ *   - Limit: with W the split count after planning (num_splits, or the planned count for
+ *     0, at most the number of tiles) and rows = batch * num_kv_heads, the partials take
+ *     round_up_256((rows + W) * G * head_dim_v * 4) + (rows + W) * G * 2 * 4 bytes.  A
+ *     problem that needs more than VX_NOALLOC_SCRATCH_BYTES is rejected with
+ *     VX_ERR_WORKSPACE and a message; pass fewer splits or use vx_sparse_decode with your
+ *     own workspace.
+ *   - Set-up and memory: the array is placed in device memory when the part of the
+ *     library that holds it is loaded on a device.  Under CUDA's default lazy module
+ *     loading that is the first call of this function on the device, which therefore
+ *     needs VX_NOALLOC_SCRATCH_BYTES of free device memory; the same call looks the
+ *     array's device address up (cudaGetSymbolAddress, with that device current; again
+ *     after a device reset).  A caller that reserves all free memory for its KV pool
+ *     makes one call on each device before reserving it (or sets
+ *     CUDA_MODULE_LOADING=EAGER), and makes that first call before any stream capture.
  *   - Sharing: every call on a device uses the same array, which keeps whatever the last
  *     call left in it; nothing in it has to start at zero (a call writes each partial
  *     before reading it).  Calls that overlap on the GPU (two streams, or two host

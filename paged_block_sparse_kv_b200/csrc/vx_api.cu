@@ -106,17 +106,22 @@ vx_status check_ptr(const void *p, const char *name, bool can_be_null = false) {
 
 // ------------------------------------------------------------------ device facts
 
+// SM count per device ordinal, looked up once; several host threads may race to fill an
+// entry, and they all store the same value.
 int sm_count_current(int *out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-    static int cache[64] = {0};
-    if (dev < 64 && cache[dev]) {
-        *out = cache[dev];
-        return 0;
+    static std::atomic<int> cache[64];
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *out = c;
+            return 0;
+        }
     }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return -1;
-    if (dev < 64) cache[dev] = n;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
     *out = n;
     return 0;
 }
@@ -420,6 +425,45 @@ vx_status decode_partial_bytes(const vx_geometry *geo, int32_t max_pages, int32_
 vx_status set_error(vx_status s, const char *msg) {
     g_last_error = msg;
     return s;
+}
+
+vx_status compact_partial_bytes(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits,
+                                size_t *bytes) {
+    VX_TRY(check_geometry(geo));
+    VX_TRY(check_max_pages(geo, max_pages));
+    VX_TRY(check_k_mode(k, 0));
+    Plan p;
+    VX_TRY(plan(geo, k, num_splits, &p));
+    const size_t slots = (size_t)(p.rows + p.chunks);
+    *bytes = up256(slots * p.G * geo->head_dim_v * sizeof(float)) + slots * p.G * 2 * sizeof(float);
+    return VX_OK;
+}
+
+vx_status sparse_decode_compact(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                                const void *k_cache, const void *v_cache, const int32_t *sel, int32_t k,
+                                float sm_scale, int32_t num_splits, void *out, float *lse, void *partials,
+                                size_t partial_bytes, int32_t *err, cudaStream_t stream) {
+    VX_TRY(check_geo(geo, table));
+    VX_TRY(check_ptr(q, "q"));
+    VX_TRY(check_ptr(k_cache, "k_cache"));
+    if (!geo->mla_shared_kv) VX_TRY(check_ptr(v_cache, "v_cache"));
+    VX_TRY(check_ptr(sel, "sel"));
+    VX_TRY(check_ptr(out, "out"));
+    VX_TRY(check_ptr(lse, "lse", true));
+    VX_TRY(check_k_mode(k, 0));
+    if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
+    if (!std::isfinite(sm_scale)) return fail(VX_ERR_INVALID_ARG, "sm_scale must be finite");
+    Plan p;
+    VX_TRY(plan(geo, k, num_splits, &p));
+    const size_t slots = (size_t)(p.rows + p.chunks);
+    WsLayout l{};
+    l.o_part = 0;
+    l.ml_part = up256(slots * p.G * geo->head_dim_v * sizeof(float));
+    l.total = l.ml_part + slots * p.G * 2 * sizeof(float);
+    if (!partials || !al16(partials)) return fail(VX_ERR_WORKSPACE, "partial buffer is NULL or not 16-byte aligned");
+    if (partial_bytes < l.total)
+        return fail(VX_ERR_WORKSPACE, "partial buffer of %zu bytes < %zu needed", partial_bytes, l.total);
+    return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, partials, out, lse, err, stream, false);
 }
 
 }  // namespace vx

@@ -144,6 +144,17 @@ vx_status decode_partial_bytes(const vx_geometry *geo, int32_t max_pages, int32_
                                size_t *bytes);
 // Set the message vx_last_error() returns on this host thread; returns s.
 vx_status set_error(vx_status s, const char *msg);
+// Bytes of split partials of the sparse decode with the partials packed alone (outputs
+// [rows + W][G][Dv] fp32, rounded up to 256 bytes, then (max, sum) [rows + W][G][2] fp32),
+// W = the resolved split count.  Validates the geometry.
+vx_status compact_partial_bytes(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits,
+                                size_t *bytes);
+// The sparse decode (same validation and kernels as vx_sparse_decode) with its split
+// partials in `partials`, laid out as compact_partial_bytes describes.
+vx_status sparse_decode_compact(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                                const void *k_cache, const void *v_cache, const int32_t *sel, int32_t k,
+                                float sm_scale, int32_t num_splits, void *out, float *lse, void *partials,
+                                size_t partial_bytes, int32_t *err, cudaStream_t stream);
 
 // Launch with programmatic dependent launch enabled when `pdl` (the kernel must call
 // pdl_wait() before reading what the previous kernel on the stream wrote).

@@ -31,6 +31,11 @@ def test_header_declares_the_binding_exports():
     assert _declared() == sorted(vx.EXPORTS)
 
 
+def test_noalloc_scratch_size_matches_the_header():
+    m = re.search(r"#define VX_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", open(HEADER).read())
+    assert m and int(m.group(1)) << int(m.group(2)) == vx.NOALLOC_SCRATCH_BYTES
+
+
 def test_library_exports_every_declared_symbol(L):
     out = subprocess.run(["nm", "-D", "--defined-only", vx.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout

@@ -10,10 +10,11 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(config, env_extra=None):
+def _run(config, env_extra=None, gpus=1):
     env = dict(os.environ, **(env_extra or {}))
     return subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
-                           "--config", config], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+                           "--config", config, "--gpus", str(gpus)], cwd=ROOT, env=env, capture_output=True,
+                          text=True, timeout=600)
 
 
 @pytest.mark.parametrize("config", ["qwen3_1p7b_gqa_b32", "mla_576_512_b16", "cont_batch_b256"])
@@ -30,6 +31,14 @@ def test_reference_arm_prints_its_line(config):
 
 
 def test_reference_arm_is_silent_on_other_ranks():
-    r = _run("qwen3_1p7b_gqa_b32", {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    r = _run("qwen3_1p7b_gqa_b32", {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, gpus=2)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_gpus_must_match_the_launched_processes():
+    # --gpus 2 in a single process (no torchrun) is refused instead of silently running one GPU
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--steps", "1", "--warmup", "0"], cwd=ROOT,
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "torchrun" in r.stderr

@@ -167,8 +167,15 @@ def test_mla_rope_aware_vs_rope_unaware_selection():
     L = w.seq_lens.cpu().numpy()
     P, k = spec.page_size, spec.k
     sels = {}
+    hq = synth.bits(w.q)
+    ptr, idx = w.page_ptr.cpu().numpy(), w.page_indices.cpu().numpy()
+    gc = synth.bits(cen)
     for dims in (0, 512):
         s = gpu_scores(w, cen, score_dims=dims)
+        # the scores themselves, every request of the full-size draw, against the oracle on the
+        # same stored centroids and the same dims
+        s_orc = oracle.scores(hq, ptr, idx, L, P, w.max_pages, 1, centroids_bf16=gc, score_dims=dims)
+        check_scores(s, s_orc, L, P)
         sel = gpu_topk(w, s)
         assert np.array_equal(sel.cpu().numpy(), oracle.topk_exact(s.cpu().numpy().astype(np.float64), L, P, k))
         sels[dims] = sel.cpu().numpy()

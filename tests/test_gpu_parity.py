@@ -222,14 +222,25 @@ def test_bad_page_id_and_length_set_the_error_word():
     assert torch.isfinite(out_ok.float()).all()
 
 
-def test_rope_unaware_score_dims():
-    w = workload("qwen_shape_small_batch")
+@pytest.mark.parametrize("name,dims", [("qwen_shape_small_batch", 64), ("mla_16heads", 512), ("mla_5heads_ragged", 512),
+                                       ("mla_page32", 512), ("mla_16heads", 64)])
+def test_rope_unaware_score_dims(name, dims):
+    """Scores on the first `dims` dims only (MLA: the 512 latent dims without the 64 rope dims, the
+    rope-unaware routing of the MLA experiment) against the oracle scoring the same stored
+    centroids on the same dims."""
+    w = workload(name)
     h = host(w)
+    P = w.spec.page_size
     cen = gpu_centroids(w)
-    s = gpu_scores(w, cen, score_dims=64)
-    s_orc = oracle.scores(h["q"], h["ptr"], h["idx"], h["L"], 16, w.max_pages, 8, centroids_bf16=synth.bits(cen),
-                          score_dims=64)
-    check_scores(s, s_orc, h["L"], 16)
+    s = gpu_scores(w, cen, score_dims=dims)
+    s_orc = oracle.scores(h["q"], h["ptr"], h["idx"], h["L"], P, w.max_pages, w.spec.num_kv_heads,
+                          centroids_bf16=synth.bits(cen), score_dims=dims)
+    check_scores(s, s_orc, h["L"], P)
+    # the cut matters: the full-dims scores differ from these on some page
+    s_full = oracle.scores(h["q"], h["ptr"], h["idx"], h["L"], P, w.max_pages, w.spec.num_kv_heads,
+                           centroids_bf16=synth.bits(cen))
+    fin = np.isfinite(s_full)
+    assert np.max(np.abs(s_full[fin] - s_orc[fin])) > 1e-3 * np.max(np.abs(s_full[fin]))
 
 
 # vx_block_topk_decode_persistent's counters: a fixed region at the head of the workspace
