@@ -36,27 +36,31 @@ L2_BYTES = 126 * 1024 * 1024
 DEFAULT_CONFIG = "qwen3_1p7b_gqa_b32"
 
 # DRAM traffic of the dominant kernel from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
-# as a multiple of the algorithmic bytes of the captured launch; valid only for the kernel source it was
-# taken on (sha256 of the file), otherwise the bench reports null.
-DECODE_TRAFFIC = {
-    "csrc/k_decode.cu": {"sha256": "cef6966877baae394024ef4d58b68199d4fad86380a21263ed1f79e472919f42",
-                         "ratio": (67.243776 + 1.478144) / 67.097856, "workload": "qwen3_1p7b_gqa_b32",
-                         "note": "captured at batch 8 (67.1 MB), scaled to the full launch by its bytes"},
-    "csrc/k_decode_mla.cu": {"sha256": "f4bb76c122e394136f340b174b39b6fa507b91f1c215d14781b44231915e6def",
-                             "ratio": (38.131456 + 0.141824) / 38.264896, "workload": "mla_576_512_b16",
-                             "note": "captured on the full workload (38.3 MB)"},
-}
+# as a multiple of the algorithmic bytes of the captured launch, per (kernel source, workload); valid only
+# for the kernel source it was taken on (sha256 of the file), otherwise the bench reports null.
+DECODE_TRAFFIC = [
+    {"file": "csrc/k_decode.cu", "sha256": "cef6966877baae394024ef4d58b68199d4fad86380a21263ed1f79e472919f42",
+     "ratio": (67.243776 + 1.478144) / 67.097856, "workload": "qwen3_1p7b_gqa_b32",
+     "note": "captured at batch 8 (67.1 MB), scaled to the full launch by its bytes"},
+    {"file": "csrc/k_decode.cu", "sha256": "cef6966877baae394024ef4d58b68199d4fad86380a21263ed1f79e472919f42",
+     "ratio": (33.705472 + 0.0064) / 33.5872, "workload": "long_ctx_128k_b8",
+     "note": "captured at batch 2 (33.6 MB), scaled to the full launch by its bytes"},
+    {"file": "csrc/k_decode.cu", "sha256": "cef6966877baae394024ef4d58b68199d4fad86380a21263ed1f79e472919f42",
+     "ratio": (134.756864 + 3.18464) / 134.485186, "workload": "cont_batch_b256",
+     "note": "captured at batch 32 (134.5 MB), scaled to the full launch by its bytes"},
+]
 
 
 def measured_traffic(kernel_file, workload, algorithmic_bytes):
     import hashlib
-    entry = DECODE_TRAFFIC.get(kernel_file)
     path = os.path.join(ROOT, "paged_block_sparse_kv_b200", kernel_file)
-    if entry is None or entry["workload"] != workload or not os.path.exists(path):
+    if not os.path.exists(path):
         return None
-    if hashlib.sha256(open(path, "rb").read()).hexdigest() != entry["sha256"]:
-        return None
-    return int(entry["ratio"] * algorithmic_bytes)
+    sha = hashlib.sha256(open(path, "rb").read()).hexdigest()
+    for entry in DECODE_TRAFFIC:
+        if entry["file"] == kernel_file and entry["workload"] == workload and entry["sha256"] == sha:
+            return int(entry["ratio"] * algorithmic_bytes)
+    return None
 
 
 def parse():
@@ -205,10 +209,19 @@ def job_throughput(batch_per_rank, ms_per_step, world):
 
 # ------------------------------------------------------------------ our arm
 
+def progress(rank, t0, what, errs=None):
+    """One line per bench phase on stderr (rank 0): wall seconds since start and, when given,
+    the device error words so far."""
+    if rank == 0:
+        extra = "" if errs is None else f" device errors {errs}"
+        print(f"[bench] {time.time() - t0:7.1f} s  {what}{extra}", file=sys.stderr, flush=True)
+
+
 def run_vx(args, rank, world, local_rank):
     import numpy as np
     import torch
     import torch.distributed as dist
+    t_start = time.time()
 
     from paged_block_sparse_kv_b200 import synth, vx
 
@@ -245,13 +258,19 @@ def run_vx(args, rank, world, local_rank):
         return cen
 
     def fused(c):
-        if c["append"]:
-            vx.vx_centroid_update(c["geo"], c["tab"], c["w"].k_cache, c["cen"], v_cache=c["w"].v_cache,
-                                  k_new=c["k_new"], v_new=c["v_new"], err=c["err"])
         if args.persistent:
+            if c["append"]:
+                vx.vx_centroid_update(c["geo"], c["tab"], c["w"].k_cache, c["cen"], v_cache=c["w"].v_cache,
+                                      k_new=c["k_new"], v_new=c["v_new"], err=c["err"])
             vx.vx_block_topk_decode_persistent(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"],
                                                k, c["out"], c["ws"], lse=c["lse"], scores_out=c["scores"],
                                                sel_out=c["sel"], err=c["err"])
+            return
+        if c["append"]:  # one call: the append, then the chained step
+            vx.vx_block_topk_decode_append(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"],
+                                           c["k_new"], c["v_new"], k, c["out"], c["ws"], lse=c["lse"], mode=mode,
+                                           seed=0, num_splits=args.splits, score_dims=args.score_dims,
+                                           scores_out=c["scores"], sel_out=c["sel"], err=c["err"])
             return
         vx.vx_block_topk_decode(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"], k, c["out"],
                                 c["ws"], lse=c["lse"], mode=mode, seed=0, num_splits=args.splits,
@@ -267,6 +286,7 @@ def run_vx(args, rank, world, local_rank):
                        seq_lens=w.seq_lens, **buffers(w, geo)))
         fused(st[0])
         torch.cuda.synchronize()
+        progress(rank, t_start, "first step", [int(st[0]["err"].item())])
         total0 = step_bytes(w, st[0]["sel"], w.seq_lens, k)[0]
         # the other copies' bytes between two uses of one copy exceed 3x L2
         n_copies = args.copies or max(2, math.floor(3 * L2_BYTES / max(total0, 1)) + 2)
@@ -296,9 +316,11 @@ def run_vx(args, rank, world, local_rank):
     # kernels per step: the centroid append (continuous batching), then the fused call's own
     # (scores, top-k, attention, merge; the persistent entry is one kernel)
     launches_per_step = (1 if args.persistent else 4) + (1 if st[0]["append"] else 0)
+    progress(rank, t_start, f"{len(st)} input copies ready")
     for c in st:
         fused(c)
     torch.cuda.synchronize()
+    progress(rank, t_start, "one step per copy", sorted(set(int(c["err"].item()) for c in st)))
     per_copy = [step_bytes(c["w"], c["sel"], c["seq_lens"], k) for c in st]
 
     stream = torch.cuda.Stream(device=dev)
@@ -343,6 +365,7 @@ def run_vx(args, rank, world, local_rank):
     gpu_id = _gpu_id(local_rank)
     with ClockSampler(gpu_id, enabled=not args.no_clocks and rank == 0) as clk:
         ms_total, (g_full, chunk) = timed_replay(fused, args.steps, args.warmup)
+        progress(rank, t_start, f"timed steps: {ms_total / args.steps * 1e3:.2f} us per step")
         # keep the GPU in the same steady state for >= 1 s so the sampler sees it
         t_end = time.time() + 1.0
         while time.time() < t_end:
@@ -353,6 +376,7 @@ def run_vx(args, rank, world, local_rank):
 
     # per-step distribution of the appending loop (mean and median over its steps): one graph per
     # step, replayed back to back with an event between steps (so no overlap across steps)
+    progress(rank, t_start, "clock sampling done")
     per_step = None
     if spec.steps:
         import numpy as np
@@ -383,6 +407,7 @@ def run_vx(args, rank, world, local_rank):
                             c["ws"], lse=c["lse"], num_splits=args.splits, err=c["err"])
     dec_steps = max(len(st), min(args.steps, 1000))
     ms_dec, _ = timed_replay(decode_only, dec_steps, 3)
+    progress(rank, t_start, f"sparse decode call: {ms_dec / dec_steps * 1e3:.2f} us")
     ms_dec_launch = ms_dec / dec_steps
     dec_bytes = sum(p[1] for p in per_copy) / len(per_copy)
     dec_gbs = dec_bytes / (ms_dec_launch * 1e-3) / 1e9
@@ -406,6 +431,7 @@ def run_vx(args, rank, world, local_rank):
                          ("chain", chain)):
             ms_b, _ = timed_replay(fn, nb, 3)
             breakdown[name + "_us"] = round(ms_b / nb * 1e3, 3)
+            progress(rank, t_start, f"breakdown {name}: {breakdown[name + '_us']} us")
         if spec.steps:
             def append_only(c):
                 vx.vx_centroid_update(c["geo"], c["tab"], c["w"].k_cache, c["cen"], v_cache=c["w"].v_cache,
@@ -506,6 +532,7 @@ def run_vx(args, rank, world, local_rank):
         assert torch.equal(S["h_out"].to(dev), S["d_out"]), "e2e: the D2H copy does not hold the call's outputs"
 
     errs = [int(c["err"].item()) for c in st]
+    progress(rank, t_start, f"e2e: {ms_e2e * 1e3:.2f} us per step", sorted(set(errs)))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -521,7 +548,8 @@ def run_vx(args, rank, world, local_rank):
                        "head_dim_v": spec.head_dim_v, "page_size": spec.page_size, "k_pages": k,
                        "context": list(spec.ctx), "topk_mode": args.mode, "splits": args.splits or "planned",
                        "score_dims": args.score_dims or spec.head_dim_qk,
-                       "entry": "vx_block_topk_decode_persistent" if args.persistent else "vx_block_topk_decode",
+                       "entry": "vx_block_topk_decode_persistent" if args.persistent else (
+                           "vx_block_topk_decode_append" if st[0]["append"] else "vx_block_topk_decode"),
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": l2_note.format(n=len(st), mb=mean_bytes * max(1, len(st) - 1) / 1e6)},
             "hbm": {"roofline_bytes_per_step": int(mean_bytes), "achieved_gbs": round(step_gbs, 1),

@@ -194,6 +194,25 @@ vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *tabl
                                int32_t *err, void *stream);
 
 /*
+ * One continuous-batching decode step: every request appends one token and then decodes
+ * (paper note, 系统设计 1: the cache stage keeps each page's centroid as tokens arrive;
+ * 系统设计 3: fusion of the sequence-local steps).  The append of vx_centroid_update
+ * (k_new, first_pos NULL) runs first: each request's new token (k_new [B][Hkv][Dqk],
+ * v_new [B][Hkv][Dv], v_new ignored for MLA) goes into slot (seq_lens[b]-1) % P of its
+ * page, whose centroid is recomputed from its keys; seq_lens already counts the new token
+ * and its page is installed in the table.  Then vx_block_topk_decode's score -> top-k ->
+ * attention chain runs on the same stream, its first kernel launched with programmatic
+ * dependent launch behind the append, so it starts while the append drains.  Arguments
+ * and results as in vx_centroid_update plus vx_block_topk_decode; same workspace size.
+ */
+vx_status vx_block_topk_decode_append(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                                      void *k_cache, void *v_cache, void *centroids, const void *k_new,
+                                      const void *v_new, int32_t k, int32_t mode, uint64_t seed,
+                                      float sm_scale, int32_t score_dims, int32_t num_splits, void *out,
+                                      float *lse, float *scores_out, int32_t *sel_out, void *ws,
+                                      size_t ws_bytes, int32_t *err, void *stream);
+
+/*
  * The same decode step (exact top-k, full score dims) as ONE persistent kernel (paper note,
  * 系统设计 3: fusion and workload planning, taken to a single launch).  Its warps take work
  * items from two ticket counters: score a span of one request's pages, attend a span of

@@ -143,6 +143,9 @@ __global__ void __launch_bounds__(CEN_WARPS * 32) k_centroid_rebuild(CentroidArg
 // slot, then recomputes that page's centroid with the new row taken from k_new.
 template <int D>
 __global__ void k_centroid_append(CentroidArgs a) {
+    // a dependent scorer (vx_block_topk_decode_append) may launch now; it waits for this
+    // grid's end and writes before it reads anything
+    pdl_trigger();
     const int b = blockIdx.x;
     const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (h >= a.Hkv) return;

@@ -3,7 +3,7 @@
 // Host validation runs before anything is launched and touches no CUDA state, so bad
 // arguments fail the same way with or without a GPU.  Workload planning (paper note,
 // section 系统设计 3) picks the split count from the SM count: one persistent block of
-// DEC_WARPS worker warps per SM for GQA, two blocks per SM for MLA.
+// DEC_WARPS worker warps per SM for GQA, one tensor-core CTA per SM for MLA.
 #include <cudaTypedefs.h>
 
 #include <cmath>
@@ -60,7 +60,7 @@ vx_status check_geometry(const vx_geometry *g) {
         if (g->num_kv_heads != 1 || g->head_dim_qk != 576 || g->head_dim_v != 512)
             return fail(VX_ERR_UNSUPPORTED, "MLA geometry must be 1 KV head, head_dim_qk 576, head_dim_v 512");
         if (G > 16) return fail(VX_ERR_UNSUPPORTED, "MLA supports at most 16 query heads (got %d)", G);
-        if (g->page_size % vx::MLA_TILE_TOKENS)
+        if (g->page_size % vx::MLA_MIN_PAGE)
             return fail(VX_ERR_UNSUPPORTED, "MLA page_size must be 32 or 64 (got %d)", g->page_size);
     } else {
         if (g->head_dim_qk != g->head_dim_v) return fail(VX_ERR_UNSUPPORTED, "GQA needs head_dim_qk == head_dim_v");
@@ -135,20 +135,19 @@ struct Plan {
     bool mla;
 };
 
-constexpr int MLA_BLOCKS_PER_SM = 2;
 
 vx_status plan(const vx_geometry *g, int32_t k, int32_t num_splits, Plan *p) {
     p->mla = g->mla_shared_kv != 0;
     p->G = g->num_q_heads / g->num_kv_heads;
     p->rows = (int64_t)g->batch * g->num_kv_heads;
-    p->tiles_per_page = g->page_size / (p->mla ? vx::MLA_TILE_TOKENS : vx::DEC_TILE);
+    p->tiles_per_page = g->page_size / (p->mla ? std::min(g->page_size, vx::MLA_TILE_ROWS) : vx::DEC_TILE);
     p->units_per_row = (int64_t)k * p->tiles_per_page;
     p->units = p->rows * p->units_per_row;
     int64_t w = num_splits;
     if (w <= 0) {
         int sms = 0;
         if (sm_count_current(&sms) != 0) return fail(VX_ERR_CUDA, "cannot query the current device's SM count");
-        w = p->mla ? (int64_t)sms * MLA_BLOCKS_PER_SM : (int64_t)sms * vx::DEC_WARPS;
+        w = p->mla ? (int64_t)sms : (int64_t)sms * vx::DEC_WARPS;  // MLA: one CTA per SM
     }
     if (w > p->units) w = p->units;
     if (w < 1) w = 1;
@@ -266,19 +265,17 @@ vx_status make_cache_map(CUtensorMap *map, const void *ptr, int dim, int page_si
     return VX_OK;
 }
 
-// Whole token rows in one copy: the row of `dim` bf16 values is viewed as dim / 64 blocks
-// of 64 columns (128 bytes, the 128-byte swizzle span), so a box of (64, dim / 64,
-// box_rows, 1) lands box_rows full rows in shared memory as consecutive 128-byte segments
-// (segment = row * (dim / 64) + block), each swizzled by its segment index.
-vx_status make_cache_map_rows(CUtensorMap *map, const void *ptr, int dim, int page_size, int64_t page_heads,
-                              int box_rows) {
+// The query rows [batch * Hq][dim] as (64 columns, rows, dim / 64 blocks): a box of 16 rows
+// lands as dim / 64 blocks of 16 rows x 128 bytes (128-byte swizzle), the layout of a
+// K-major tensor-core operand with 16 rows.  Rows past the end read as zero.
+vx_status make_query_map(CUtensorMap *map, const void *ptr, int dim, int64_t rows) {
     auto fn = encode_fn();
     if (!fn) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    cuuint64_t gdim[4] = {64, (cuuint64_t)(dim / 64), (cuuint64_t)page_size, (cuuint64_t)page_heads};
-    cuuint64_t gstride[3] = {128, (cuuint64_t)dim * 2, (cuuint64_t)dim * 2 * page_size};
-    cuuint32_t box[4] = {64, (cuuint32_t)(dim / 64), (cuuint32_t)box_rows, 1};
-    cuuint32_t estride[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), gdim, gstride, box, estride,
+    cuuint64_t gdim[3] = {64, (cuuint64_t)rows, (cuuint64_t)(dim / 64)};
+    cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, 128};
+    cuuint32_t box[3] = {64, 16, (cuuint32_t)(dim / 64)};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), gdim, gstride, box, estride,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(VX_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -339,9 +336,11 @@ vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q,
     const int64_t page_heads = g->num_pool_pages * g->num_kv_heads;
     cudaError_t e;
     if (p.mla) {
-        CUtensorMap tmK;
-        VX_TRY(make_cache_map_rows(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::MLA_TILE_TOKENS));
-        e = vx::launch_decode_mla(a, tmK, p.grid, s, pdl);
+        CUtensorMap tmK, tmQ;
+        VX_TRY(make_cache_map_blocks(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads,
+                                     g->page_size / p.tiles_per_page));
+        VX_TRY(make_query_map(&tmQ, q, g->head_dim_qk, (int64_t)g->batch * g->num_q_heads));
+        e = vx::launch_decode_mla(a, tmK, tmQ, p.grid, s, pdl);
     } else {
         CUtensorMap tmK, tmV;
         VX_TRY(make_cache_map_blocks(&tmK, k_cache, g->head_dim_qk, g->page_size, page_heads, vx::DEC_TILE));
@@ -600,11 +599,18 @@ vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, c
                      static_cast<cudaStream_t>(stream), false);
 }
 
-vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *table, const void *q, const void *k_cache,
-                               const void *v_cache, const void *centroids, int32_t k, int32_t mode, uint64_t seed,
-                               float sm_scale, int32_t score_dims, int32_t num_splits, void *out, float *lse,
-                               float *scores_out, int32_t *sel_out, void *ws, size_t ws_bytes, int32_t *err,
-                               void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The chained step score -> top-k -> decode -> merge; `append` (k_new non-NULL) first writes
+// each request's new token and recomputes its page's centroid, and the scorer then follows
+// with programmatic dependent launch.
+vx_status fused_step(const vx_geometry *geo, const vx_page_table *table, const void *q, const void *k_cache,
+                     const void *v_cache, const void *centroids, void *k_cache_w, void *v_cache_w, void *centroids_w,
+                     const void *k_new, const void *v_new, int32_t k, int32_t mode, uint64_t seed, float sm_scale,
+                     int32_t score_dims, int32_t num_splits, void *out, float *lse, float *scores_out, int32_t *sel_out,
+                     void *ws, size_t ws_bytes, int32_t *err, void *stream) {
     VX_TRY(check_geo(geo, table));
     VX_TRY(check_ptr(q, "q"));
     VX_TRY(check_ptr(k_cache, "k_cache"));
@@ -624,14 +630,68 @@ vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *tabl
     if (!ws || !al16(ws)) return fail(VX_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
     if (ws_bytes < l.total)
         return fail(VX_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, l.total);
+    if (k_new) {
+        VX_TRY(check_ptr(k_new, "k_new"));
+        if (!geo->mla_shared_kv) VX_TRY(check_ptr(v_new, "v_new"));
+    }
     float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<char *>(ws) + l.scores);
     int32_t *sel = sel_out ? sel_out : reinterpret_cast<int32_t *>(static_cast<char *>(ws) + l.sel);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = vx::launch_score(score_args(geo, table, q, centroids, score_dims, scores, err), s, false);
+    cudaError_t e;
+    if (k_new) {
+        vx::CentroidArgs ca{};
+        ca.page_ptr = table->page_ptr;
+        ca.page_indices = table->page_indices;
+        ca.seq_lens = table->seq_lens;
+        ca.first_pos = nullptr;
+        ca.k_cache = k_cache_w;
+        ca.v_cache = v_cache_w;
+        ca.centroids = centroids_w;
+        ca.k_new = k_new;
+        ca.v_new = v_new;
+        ca.err = err;
+        ca.B = geo->batch;
+        ca.Hkv = geo->num_kv_heads;
+        ca.Dqk = geo->head_dim_qk;
+        ca.Dv = geo->head_dim_v;
+        ca.P = geo->page_size;
+        ca.max_pages = table->max_pages;
+        ca.mla_shared_kv = geo->mla_shared_kv;
+        ca.num_pool_pages = geo->num_pool_pages;
+        e = vx::launch_centroid(ca, vx::CEN_APPEND, s);
+        if (e != cudaSuccess) return cuda_fail(e, "centroid append launch");
+    }
+    // the scorer reads nothing before its dependency wait, so it may always launch early
+    e = vx::launch_score(score_args(geo, table, q, centroids, score_dims, scores, err), s, true);
     if (e != cudaSuccess) return cuda_fail(e, "score launch");
     e = vx::launch_topk(topk_args(geo, table, scores, k, seed, sel, err), mode, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
     return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, ws, out, lse, err, s, true);
+}
+
+}  // namespace
+
+extern "C" {
+
+vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *table, const void *q, const void *k_cache,
+                               const void *v_cache, const void *centroids, int32_t k, int32_t mode, uint64_t seed,
+                               float sm_scale, int32_t score_dims, int32_t num_splits, void *out, float *lse,
+                               float *scores_out, int32_t *sel_out, void *ws, size_t ws_bytes, int32_t *err,
+                               void *stream) {
+    return fused_step(geo, table, q, k_cache, v_cache, centroids, nullptr, nullptr, nullptr, nullptr, nullptr, k, mode,
+                      seed, sm_scale, score_dims, num_splits, out, lse, scores_out, sel_out, ws, ws_bytes, err,
+                      stream);
+}
+
+vx_status vx_block_topk_decode_append(const vx_geometry *geo, const vx_page_table *table, const void *q,
+                                      void *k_cache, void *v_cache, void *centroids, const void *k_new,
+                                      const void *v_new, int32_t k, int32_t mode, uint64_t seed, float sm_scale,
+                                      int32_t score_dims, int32_t num_splits, void *out, float *lse, float *scores_out,
+                                      int32_t *sel_out, void *ws, size_t ws_bytes, int32_t *err, void *stream) {
+    if (!k_new) return fail(VX_ERR_INVALID_ARG, "k_new is NULL (use vx_block_topk_decode for a step without append)");
+    return fused_step(geo, table, q, k_cache, v_cache, centroids, k_cache, v_cache, centroids, k_new, v_new, k, mode,
+                      seed, sm_scale, score_dims, num_splits, out, lse, scores_out, sel_out, ws, ws_bytes, err,
+                      stream);
 }
 
 vx_status vx_block_topk_decode_persistent(const vx_geometry *geo, const vx_page_table *table, const void *q,

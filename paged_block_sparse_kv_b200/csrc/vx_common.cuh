@@ -87,6 +87,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, unsigned parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread may sleep (issuing nothing) for up to about
+// `hint_ns` nanoseconds, and is woken when the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, unsigned parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 // Wait for phase `parity` of the barrier to complete, for at most about WAIT_LIMIT_NS.
 // Short waits spin on the non-blocking test_wait (a data tile usually lands within a
 // microsecond); longer ones fall back to try_wait, which may suspend the thread, and

@@ -26,7 +26,8 @@ constexpr int APPROX_BITS_COARSE = 8;    // approximate top-k, mode 3: 256 codes
 constexpr int DEC_WARPS = 8;             // GQA decode: worker warps per block
 constexpr int DEC_STAGES = 3;            // GQA decode: 16-token tiles in flight per warp
 constexpr int DEC_TILE = 16;             // GQA decode: tokens per tile (one mma M or K step)
-constexpr int MLA_TILE_TOKENS = 32;      // MLA decode: tokens per tile
+constexpr int MLA_MIN_PAGE = 32;         // MLA decode: pages of 32 or 64 tokens
+constexpr int MLA_TILE_ROWS = 64;        // MLA decode: tokens per tile (a page of up to 64 tokens)
 
 // ------------------------------------------------------------------ argument blocks
 struct TableArgs {
@@ -130,8 +131,9 @@ cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s, bool pdl);
 cudaError_t launch_topk(const TopkArgs &a, int mode, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_gqa(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                               int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_decode_mla(const DecodeArgs &a, const CUtensorMap &tmK, int grid, cudaStream_t s,
-                              bool pdl);
+// grid = split count (one CTA per split); tmQ views q as (64 columns, rows = batch * Hq, 9 blocks)
+cudaError_t launch_decode_mla(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmQ, int grid,
+                              cudaStream_t s, bool pdl);
 cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s, bool pdl);
 // grid = SM count (one block of FUSED_WARPS warps per SM)
 cudaError_t launch_fused(const FusedArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV, cudaStream_t s);

@@ -23,7 +23,8 @@ NOALLOC_SCRATCH_BYTES = 16 << 20  # VX_NOALLOC_SCRATCH_BYTES of include/vx.h
 
 # every symbol include/vx.h declares
 EXPORTS = ["vx_centroid_update", "vx_score_pages", "vx_topk_pages", "vx_sparse_decode",
-           "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_block_topk_decode_persistent", "vx_workspace_size", "vx_planned_splits", "vx_status_string",
+           "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_block_topk_decode_append",
+           "vx_block_topk_decode_persistent", "vx_workspace_size", "vx_planned_splits", "vx_status_string",
            "vx_last_error", "vx_version"]
 
 
@@ -65,6 +66,8 @@ def lib():
         L.vx_block_topk_decode_persistent.argtypes = [G, T, p, p, p, p, i32, f32, p, p, p, p, p, sz, p, p]
         L.vx_block_topk_decode.argtypes = [G, T, p, p, p, p, i32, i32, u64, f32, i32, i32, p, p, p, p, p, sz,
                                            p, p]
+        L.vx_block_topk_decode_append.argtypes = [G, T, p, p, p, p, p, p, i32, i32, u64, f32, i32, i32, p, p, p, p,
+                                                  p, sz, p, p]
         L.vx_workspace_size.argtypes = [G, i32, i32, i32]
         L.vx_workspace_size.restype = sz
         L.vx_planned_splits.argtypes = [G, i32, i32]
@@ -74,7 +77,8 @@ def lib():
         L.vx_last_error.restype = ctypes.c_char_p
         L.vx_version.restype = ctypes.c_char_p
         for name in ("vx_centroid_update", "vx_score_pages", "vx_topk_pages", "vx_sparse_decode",
-                     "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_block_topk_decode_persistent"):
+                     "vx_sparse_decode_noalloc", "vx_block_topk_decode", "vx_block_topk_decode_append",
+                     "vx_block_topk_decode_persistent"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -205,6 +209,21 @@ def vx_block_topk_decode(geo: Geometry, table: PageTable, q, k_cache, v_cache, c
                                    score_dims, num_splits, _ptr(out, torch.bfloat16), _ptr(lse, torch.float32),
                                    _ptr(scores_out, torch.float32), _ptr(sel_out, torch.int32), _ptr(ws),
                                    ws.numel() * ws.element_size(), _ptr(err, torch.int32), _stream(stream)))
+
+
+def vx_block_topk_decode_append(geo: Geometry, table: PageTable, q, k_cache, v_cache, centroids, k_new, v_new,
+                                k: int, out, ws, lse=None, mode=0, seed=0, sm_scale=0.0, score_dims=0, num_splits=0,
+                                scores_out=None, sel_out=None, err=None, stream=None):
+    """One appending decode step: write each request's new token (k_new [B][Hkv][Dqk], v_new
+    [B][Hkv][Dv]) into its page and update the page centroid, then score, select and attend."""
+    _ok(lib().vx_block_topk_decode_append(ctypes.byref(geo.c()), ctypes.byref(table.c()), _ptr(q, torch.bfloat16),
+                                          _ptr(k_cache, torch.bfloat16), _ptr(v_cache, torch.bfloat16),
+                                          _ptr(centroids, torch.bfloat16), _ptr(k_new, torch.bfloat16),
+                                          _ptr(v_new, torch.bfloat16), k, mode, seed & (2 ** 64 - 1),
+                                          float(sm_scale), score_dims, num_splits, _ptr(out, torch.bfloat16),
+                                          _ptr(lse, torch.float32), _ptr(scores_out, torch.float32),
+                                          _ptr(sel_out, torch.int32), _ptr(ws), ws.numel() * ws.element_size(),
+                                          _ptr(err, torch.int32), _stream(stream)))
 
 
 def vx_block_topk_decode_persistent(geo: Geometry, table: PageTable, q, k_cache, v_cache, centroids, k: int, out,

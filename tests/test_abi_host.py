@@ -125,6 +125,20 @@ def test_bad_pointers_and_sizes(L):
                               FAKE, need, None, None) == vx.VX_ERR_INVALID_ARG
 
 
+def test_appending_step_validation(L):
+    # vx_block_topk_decode_append needs k_new (and v_new for GQA) and checks the step's arguments
+    # before any launch (explicit split count: no device query needed)
+    gp, tp = ctypes.byref(_geo()), ctypes.byref(_table())
+    f0 = ctypes.c_float(0.0)
+    args = lambda k_new, v_new, ws_bytes: (gp, tp, FAKE, FAKE, FAKE, FAKE, k_new, v_new, 4, 0, 0, f0, 0, 8, FAKE,
+                                           None, None, None, FAKE, ws_bytes, None, None)
+    assert L.vx_block_topk_decode_append(*args(None, FAKE, 1 << 30)) == vx.VX_ERR_INVALID_ARG
+    assert b"k_new" in L.vx_last_error()
+    assert L.vx_block_topk_decode_append(*args(FAKE, None, 1 << 30)) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_block_topk_decode_append(*args(FAKE + 8, FAKE, 1 << 30)) == vx.VX_ERR_INVALID_ARG  # misaligned
+    assert L.vx_block_topk_decode_append(*args(FAKE, FAKE, 16)) == vx.VX_ERR_WORKSPACE
+
+
 def test_persistent_step_validation(L):
     # vx_block_topk_decode_persistent refuses what it cannot run, before any launch
     tp = ctypes.byref(_table())

@@ -129,10 +129,10 @@ def test_continuous_batching_steps():
     for s in range(spec.steps):
         L = w.seq_lens_at(s)
         tab = table(w, L)
-        vx.vx_centroid_update(geo, tab, w.k_cache, cen, v_cache=w.v_cache, k_new=w.step_k_new[s],
-                              v_new=w.step_v_new[s], err=err)
-        vx.vx_block_topk_decode(geo, tab, w.step_q[s], w.k_cache, w.v_cache, cen, spec.k, out, ws, lse=lse,
-                                scores_out=scores, sel_out=sel, err=err)
+        # one call per step: append the new tokens (cache + tail centroids), then score, select, attend
+        vx.vx_block_topk_decode_append(geo, tab, w.step_q[s], w.k_cache, w.v_cache, cen, w.step_k_new[s],
+                                       w.step_v_new[s], spec.k, out, ws, lse=lse, scores_out=scores, sel_out=sel,
+                                       err=err)
         L_sub = L.cpu().numpy()[reqs]
         kc, vc = oracle.append(kc, vc, init["page_ptr"], init["page_indices"], L_sub,
                                synth.bits(w.step_k_new[s][ridx.to(dev)]), synth.bits(w.step_v_new[s][ridx.to(dev)]))

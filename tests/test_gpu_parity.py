@@ -154,6 +154,58 @@ def test_approx_topk_bit_exact_on_gpu_scores(name):
     assert recall(sel.cpu().numpy(), exact) > 0.5
 
 
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "mla_16heads", "g16_d64_page64", "edges_1tok_fullpage_ragged"])
+def test_fused_step_modes_match_separate_calls(name):
+    """The fused step in every top-k mode gives the separate calls' scores and selection bit for
+    bit (the chained kernels run with programmatic dependent launch)."""
+    w = workload(name)
+    cen = gpu_centroids(w)
+    s = gpu_scores(w, cen)
+    for mode in (0, 1, 2, 3):
+        for seed in (0, 77):
+            err = err_word()
+            out, lse, s_f, sel_f = gpu_fused(w, cen, mode=mode, seed=seed, err=err)
+            assert np.array_equal(s_f.cpu().numpy(), s.cpu().numpy(), equal_nan=True)
+            assert torch.equal(sel_f, gpu_topk(w, s, mode=mode, seed=seed))
+            torch.cuda.synchronize()
+            assert int(err.item()) == 0
+            if mode == 0:
+                break
+
+
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "mla_16heads", "g1_many_rows"])
+def test_fused_steps_on_a_stream_and_in_a_graph(name):
+    """Back-to-back fused steps on a created stream (where the kernels' programmatic dependent
+    launches take effect) and replayed from a CUDA graph give the default-stream result bit for
+    bit, with no device error (a bounded wait that ran out would set VX_DATA_TIMEOUT)."""
+    w = workload(name)
+    cen = gpu_centroids(w)
+    ref = gpu_fused(w, cen)
+    torch.cuda.synchronize()
+    st = torch.cuda.Stream()
+    err = err_word()
+    bufs = [workspace(w) for _ in range(2)]
+    with torch.cuda.stream(st):
+        runs = [gpu_fused(w, cen, err=err, ws=bufs[i % 2]) for i in range(6)]
+    torch.cuda.synchronize()
+    outs = []
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(st):
+        gpu_fused(w, cen, err=err, ws=bufs[0])  # warm-up before capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=st):
+            for i in range(4):
+                outs.append(gpu_fused(w, cen, err=err, ws=bufs[i % 2]))
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for r in runs + outs:
+        assert torch.equal(r[0].view(torch.int16), ref[0].view(torch.int16)) and torch.equal(r[1], ref[1])
+        assert torch.equal(r[3], ref[3])
+    del g
+
+
 def test_topk_ties_and_signed_zero():
     # crafted rows: all-equal scores pick the lowest pages; -0.0 ties with +0.0
     spec = synth.custom_spec(batch=2, num_q_heads=2, num_kv_heads=2, head_dim_qk=64, page_size=16,
@@ -195,6 +247,55 @@ def test_append_steps_match_oracle():
     assert np.array_equal(gv[used].view(np.int16), vc[used].view(np.int16))
     _, c16 = oracle.centroids(kc, ptr, idx, Lf)
     assert np.array_equal(synth.bits(cen)[used], c16[used])
+
+
+@pytest.mark.parametrize("mla", [False, True])
+def test_appending_step_equals_append_then_fused_call(mla):
+    """vx_block_topk_decode_append (append chained into the step) gives the same bits as
+    vx_centroid_update's append followed by vx_block_topk_decode, step after step: caches,
+    centroids, scores, selection, out and lse."""
+    if mla:
+        spec = synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
+                                 page_size=64, mla_shared_kv=True, ctx=("list", [63, 64, 700]), k=5, steps=4)
+    else:
+        spec = synth.custom_spec(batch=4, num_q_heads=8, num_kv_heads=4, head_dim_qk=128, page_size=16,
+                                 ctx=("list", [15, 16, 33, 1000]), k=6, steps=4)
+    runs = []
+    for fused in (False, True):
+        w = synth.make(spec, 41, "cuda")
+        geo = geometry(w)
+        cen = gpu_centroids(w)
+        ws = workspace(w)
+        err = err_word()
+        outs = []
+        for s in range(spec.steps):
+            L = w.seq_lens_at(s)
+            tab = table(w, L)
+            out = torch.empty((w.batch, spec.num_q_heads, spec.head_dim_v), dtype=torch.bfloat16, device="cuda")
+            lse = torch.empty((w.batch, spec.num_q_heads), dtype=torch.float32, device="cuda")
+            sc = torch.full((w.batch, spec.num_kv_heads, w.max_pages), float("nan"), device="cuda")
+            sel = torch.empty((w.batch, spec.num_kv_heads, spec.k), dtype=torch.int32, device="cuda")
+            v_new = None if w.step_v_new is None else w.step_v_new[s]  # MLA: the value is the latent key
+            if fused:
+                vx.vx_block_topk_decode_append(geo, tab, w.step_q[s], w.k_cache, w.v_cache, cen, w.step_k_new[s],
+                                               v_new, spec.k, out, ws, lse=lse, scores_out=sc, sel_out=sel, err=err)
+            else:
+                vx.vx_centroid_update(geo, tab, w.k_cache, cen, v_cache=w.v_cache, k_new=w.step_k_new[s],
+                                      v_new=v_new, err=err)
+                vx.vx_block_topk_decode(geo, tab, w.step_q[s], w.k_cache, w.v_cache, cen, spec.k, out, ws, lse=lse,
+                                        scores_out=sc, sel_out=sel, err=err)
+            outs.append((out, lse, sc, sel))
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        runs.append((outs, w.k_cache, w.v_cache, cen))
+    (o0, k0, v0, c0), (o1, k1, v1, c1) = runs
+    assert torch.equal(k0.view(torch.int16), k1.view(torch.int16)) and torch.equal(c0.view(torch.int16),
+                                                                                   c1.view(torch.int16))
+    if v0 is not None:
+        assert torch.equal(v0.view(torch.int16), v1.view(torch.int16))
+    for a, b in zip(o0, o1):
+        assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)) and torch.equal(a[1], b[1])
+        assert np.array_equal(a[2].cpu().numpy(), b[2].cpu().numpy(), equal_nan=True) and torch.equal(a[3], b[3])
 
 
 def test_bad_page_id_and_length_set_the_error_word():
