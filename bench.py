@@ -533,6 +533,16 @@ def run_vx(args, rank, world, local_rank):
 
     errs = [int(c["err"].item()) for c in st]
     progress(rank, t_start, f"e2e: {ms_e2e * 1e3:.2f} us per step", sorted(set(errs)))
+    # the device-timed steps once more, after the other legs (a drift here is the GPU's state,
+    # e.g. its clocks after seconds of load, not the e2e copies)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g_full.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    progress(rank, t_start, f"device steps again after e2e: {e0.elapsed_time(e1) / chunk * 1e3:.2f} us per step")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -43,11 +43,12 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Let the next grid on the stream launch now (it still waits in pdl_wait for this grid's end
 // and writes).  Only the top-k kernel triggers, late in each block: its dependent (the decode
-// kernel) then lands as top-k blocks leave and runs its prologue meanwhile.  A trigger in the
-// scorer (at its start, or once a warp has issued its last copies) measured slower: top-k
-// blocks fit beside a scorer block and then compete with it; one at the decode kernel's start
-// measured slower and one after its last loads made no difference.  Without a trigger, the
-// next grid launches at block exit.
+// kernel) lands as top-k blocks leave and runs its prologue meanwhile.  Measured without
+// gain: a trigger in the scorer (with many rows the top-k blocks beside a scorer block compete
+// with it, -10% on the headline step; with the MLA batch's 16 rows, 39.9 against 34.6 us per
+// step), at the GQA decode kernel's start (slower) or after its last loads, and in the MLA
+// decode kernel once its producer has issued the last copy.  Without a trigger, the next grid
+// launches at block exit.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------------- mbarrier

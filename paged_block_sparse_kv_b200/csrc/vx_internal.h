@@ -60,6 +60,10 @@ struct TopkArgs {
     const float *scores;
     int32_t *sel;
     int32_t *err;
+    // optional (sel_phys != NULL): the physical page of every chosen page, [B][Hkv][k], read
+    // from the table (page_ptr, page_indices) while the scores are still being computed
+    const int32_t *page_ptr, *page_indices;
+    int32_t *sel_phys;
     int32_t B, Hkv, P, max_pages, k, smem_keys;
     int32_t warp_max;  // exact rows of at most this many pages go to one warp (0: none)
     uint64_t seed;
@@ -67,6 +71,7 @@ struct TopkArgs {
 
 struct DecodeArgs {
     const int32_t *page_ptr, *page_indices, *seq_lens, *sel;
+    const int32_t *sel_phys;  // NULL, or the physical page of each selection slot (saves a lookup)
     const __nv_bfloat16 *q;
     float *o_part;   // [slots][G][Dv] unnormalised partial outputs
     float *ml_part;  // [slots][G][2]  (running max in log2 units, running sum)
