@@ -74,6 +74,8 @@ def parse():
     ap.add_argument("--mode", default="exact", choices=["exact", "approx", "approx1024", "approx256"],
                     help="top-k mode: exact, or approximate with 4096, 1024 or 256 codes")
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--no-table-ready", action="store_true",
+                    help="call the chained step without VX_TABLE_READY (every read waits for the previous kernel)")
     ap.add_argument("--score-dims", type=int, default=0,
                     help="dims of the key scored against the centroids (0: all; 512 on MLA: rope-unaware)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (small profiling cases only)")
@@ -234,6 +236,10 @@ def run_vx(args, rank, world, local_rank):
     if args.batch:
         spec = synth.Spec(**{**spec.__dict__, "batch": args.batch})
     mode = {"exact": 0, "approx": 1, "approx1024": 2, "approx256": 3}[args.mode]
+    # the chained steps' mode: the page tables and lengths here are set up before the timed
+    # region (or copied in by the e2e leg's own H2D copies), never written by the kernel
+    # right before a call, so the scorer may read them while that kernel finishes
+    step_mode = mode if args.no_table_ready else mode | vx.VX_TABLE_READY
     k = spec.k
     B = spec.batch
 
@@ -268,12 +274,12 @@ def run_vx(args, rank, world, local_rank):
             return
         if c["append"]:  # one call: the append, then the chained step
             vx.vx_block_topk_decode_append(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"],
-                                           c["k_new"], c["v_new"], k, c["out"], c["ws"], lse=c["lse"], mode=mode,
+                                           c["k_new"], c["v_new"], k, c["out"], c["ws"], lse=c["lse"], mode=step_mode,
                                            seed=0, num_splits=args.splits, score_dims=args.score_dims,
                                            scores_out=c["scores"], sel_out=c["sel"], err=c["err"])
             return
         vx.vx_block_topk_decode(c["geo"], c["tab"], c["q"], c["w"].k_cache, c["w"].v_cache, c["cen"], k, c["out"],
-                                c["ws"], lse=c["lse"], mode=mode, seed=0, num_splits=args.splits,
+                                c["ws"], lse=c["lse"], mode=step_mode, seed=0, num_splits=args.splits,
                                 score_dims=args.score_dims, scores_out=c["scores"], sel_out=c["sel"], err=c["err"])
 
     st = []
@@ -558,6 +564,7 @@ def run_vx(args, rank, world, local_rank):
                        "head_dim_v": spec.head_dim_v, "page_size": spec.page_size, "k_pages": k,
                        "context": list(spec.ctx), "topk_mode": args.mode, "splits": args.splits or "planned",
                        "score_dims": args.score_dims or spec.head_dim_qk,
+                       "table_ready": not (args.no_table_ready or args.persistent),
                        "entry": "vx_block_topk_decode_persistent" if args.persistent else (
                            "vx_block_topk_decode_append" if st[0]["append"] else "vx_block_topk_decode"),
                        "parallelism": f"replicas{world}" if world > 1 else "single",

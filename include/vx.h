@@ -185,7 +185,20 @@ vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, c
  * sel_out (may be NULL) receive the intermediate scores and selection; when NULL they
  * live in the workspace.  score_dims as in vx_score_pages.  ws: vx_workspace_size bytes,
  * no initial contents needed.
+ * mode: vx_topk_pages's mode (0..3), optionally OR-ed with VX_TABLE_READY.
  */
+/*
+ * Flag OR-ed into the mode of the two chained steps below.  It promises that the page table
+ * (page_ptr, page_indices) and seq_lens were not written by the last kernel launched on the
+ * stream before the call (they came from host copies, or from an earlier kernel).  The
+ * scorer then reads them, and fetches the first page ids of its range, while that kernel
+ * is still finishing; q, the centroids and the caches are still read only after it has
+ * completed.  Without the flag every read waits for it.  Results are the same either way.
+ * A call whose table or lengths the previous kernel writes must not set the flag: the scorer
+ * could read them before they are written.
+ */
+#define VX_TABLE_READY 0x100
+
 vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *table, const void *q,
                                const void *k_cache, const void *v_cache, const void *centroids,
                                int32_t k, int32_t mode, uint64_t seed, float sm_scale,
@@ -204,6 +217,7 @@ vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *tabl
  * attention chain runs on the same stream, its first kernel launched with programmatic
  * dependent launch behind the append, so it starts while the append drains.  Arguments
  * and results as in vx_centroid_update plus vx_block_topk_decode; same workspace size.
+ * mode may carry VX_TABLE_READY (the append itself never writes the table or lengths).
  */
 vx_status vx_block_topk_decode_append(const vx_geometry *geo, const vx_page_table *table, const void *q,
                                       void *k_cache, void *v_cache, void *centroids, const void *k_new,

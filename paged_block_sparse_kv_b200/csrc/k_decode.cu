@@ -48,7 +48,6 @@ __device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u,
     const int32_t L = a.seq_lens[b];
     if (L < 1 || L > a.max_pages * a.P) return rs;  // reported by the top-k kernel
     const int32_t j = a.sel[r * a.k + i];
-    const int32_t phys_sel = a.sel_phys ? a.sel_phys[r * a.k + i] : 0;  // issued with the selection
     if (j < 0) return rs;
     const int n = ceil_div(L, a.P);
     if (j >= n) {
@@ -58,7 +57,7 @@ __device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u,
     const int tok0 = j * a.P + sub * DEC_TILE;
     const int nvalid = min(DEC_TILE, L - tok0);
     if (nvalid <= 0) return rs;
-    const int32_t phys = a.sel_phys ? phys_sel : a.page_indices[a.page_ptr[b] + j];
+    const int32_t phys = a.page_indices[a.page_ptr[b] + j];
     if (phys < 0 || phys >= a.num_pool_pages) {
         set_err(a.err, VX_DATA_BAD_PAGE_ID);
         return rs;
@@ -283,6 +282,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 template <int DV, int PER, int GROUP>
 __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     pdl_wait();
+    // the next grid on the stream may land now: the decode step's last kernel is short, and a
+    // dependent that waits for it (such as the next step's scorer) gets its start-up done meanwhile
+    pdl_trigger();
     constexpr int SLICE = 32 * PER;
     constexpr int NSLICE = DV / SLICE;
     static_assert(DV % SLICE == 0 && GROUP <= 32, "merge shape");

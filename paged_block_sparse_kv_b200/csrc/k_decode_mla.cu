@@ -100,14 +100,13 @@ __device__ __forceinline__ Resolved resolve_page(const DecodeArgs &a, int64_t u,
     const int32_t L = a.seq_lens[b];
     if (L < 1 || L > a.max_pages * a.P) return rs;
     const int32_t j = a.sel[r * a.k + i];
-    const int32_t phys_sel = a.sel_phys ? a.sel_phys[r * a.k + i] : 0;  // issued with the selection
     if (j < 0) return rs;
     const int n = ceil_div(L, a.P);
     if (j >= n) {
         set_err(a.err, VX_DATA_BAD_SELECTION);
         return rs;
     }
-    const int32_t phys = a.sel_phys ? phys_sel : a.page_indices[a.page_ptr[b] + j];
+    const int32_t phys = a.page_indices[a.page_ptr[b] + j];
     if (phys < 0 || phys >= a.num_pool_pages) {
         set_err(a.err, VX_DATA_BAD_PAGE_ID);
         return rs;

@@ -77,7 +77,9 @@ __device__ __forceinline__ int score_block_scan(int v, int *tmp, int &total) {
 
 template <int D>
 __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a) {
-    pdl_wait();  // q, the table and the centroids may come from the previous kernel
+    // q and the centroids may come from the previous kernel on the stream, and so may the
+    // table and lengths unless the call rules that out (table_ready: they are read first)
+    if (!a.table_ready) pdl_wait();
     using SP = ScoreSplit<D>;
     constexpr int DPL = SP::DPL, S = SP::S, NCH = SP::NCH;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -114,6 +116,7 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         for (int s = 0; s < SCORE_STAGES; ++s) mbar_init(bar0 + 8u * s, 1);
         fence_mbar_init();
     }
+    bool bad_len = false;  // reported after the dependency wait (err may be the previous kernel's output)
     {   // per-request page prefix and row starts
         const int per = ceil_div(a.B, blockDim.x);
         const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         for (int b = b0; b < b1; ++b) {
             const int32_t L = a.seq_lens[b];
             const bool ok = L >= 1 && L <= a.max_pages * a.P;
-            if (!ok && blockIdx.x == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
+            bad_len |= !ok;
             local += ok ? ceil_div(L, a.P) : 0;
             pptr[b] = a.page_ptr[b];
         }
@@ -157,6 +160,8 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         pre_j = static_cast<int32_t>(p_begin + lane - prefix[pre_b]);
         pre_raw = a.page_indices[pptr[pre_b] + pre_j];
     }
+    if (a.table_ready) pdl_wait();
+    if (bad_len && blockIdx.x == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
 
     // ---- group-summed queries of the block's first requests, computed once per block: each
     // thread sums one (request, KV head, 8-dim chunk) over the group's heads in head order

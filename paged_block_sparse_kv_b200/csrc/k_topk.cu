@@ -9,22 +9,20 @@ namespace vx {
 template <int ABITS, int THREADS>
 __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 8) k_topk(TopkArgs a) {
     __shared__ TopkShared sh;
-    // a.smem_keys keys, rounded up to 4, then (with a.sel_phys) as many page ids
-    extern __shared__ __align__(16) uint32_t skeys[];
-    int32_t *spages = reinterpret_cast<int32_t *>(skeys + ((a.smem_keys + 3) & ~3));
-    topk_row<ABITS, THREADS>(a, blockIdx.y, blockIdx.x, sh, skeys, spages, true);
+    extern __shared__ __align__(16) uint32_t skeys[];  // a.smem_keys entries, rounded up to 4
+    topk_row<ABITS, THREADS>(a, blockIdx.y, blockIdx.x, sh, skeys, true);
 }
 
 template <int THREADS>
 static cudaError_t launch_topk_t(const TopkArgs &a, int mode, cudaStream_t s, bool pdl) {
     const dim3 grid(a.Hkv, a.B);
-    const size_t smem = sizeof(uint32_t) * (size_t)((a.smem_keys + 3) & ~3) * (a.sel_phys ? 2 : 1);
+    const size_t smem = sizeof(uint32_t) * (size_t)((a.smem_keys + 3) & ~3);  // 16-byte run reads
     auto kern = mode == 0   ? k_topk<0, THREADS>
                 : mode == 1 ? k_topk<APPROX_BITS, THREADS>
                 : mode == 2 ? k_topk<APPROX_BITS_FAST, THREADS>
                             : k_topk<APPROX_BITS_COARSE, THREADS>;
     static std::atomic<unsigned long long> done[4];
-    cudaError_t e = ensure_smem_limit(kern, (int)(2 * sizeof(uint32_t) * TOPK_SMEM_KEYS), done[mode]);
+    cudaError_t e = ensure_smem_limit(kern, (int)(sizeof(uint32_t) * TOPK_SMEM_KEYS), done[mode]);
     if (e != cudaSuccess) return e;
     return launch_k(kern, grid, dim3(THREADS), smem, s, pdl, a);
 }

@@ -212,7 +212,7 @@ FusedPlan fused_plan(const vx_geometry *g, int32_t max_pages, int32_t k) {
 // workspace layout, every region 256-byte aligned.  The fused step's sync words come first
 // at a fixed size, so their place never depends on the batch or the page count.
 struct WsLayout {
-    size_t sync, scores, sel, sel_phys, o_part, ml_part, total;
+    size_t sync, scores, sel, o_part, ml_part, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -226,8 +226,7 @@ WsLayout ws_layout(const vx_geometry *g, int32_t max_pages, int32_t k, const Pla
     l.ml_part = l.o_part + up256(slots * p.G * g->head_dim_v * sizeof(float));
     l.scores = l.ml_part + up256(slots * p.G * 2 * sizeof(float));
     l.sel = l.scores + up256((size_t)p.rows * max_pages * sizeof(float));
-    l.sel_phys = l.sel + up256((size_t)p.rows * k * sizeof(int32_t));
-    l.total = l.sel_phys + up256((size_t)p.rows * k * sizeof(int32_t));
+    l.total = l.sel + up256((size_t)p.rows * k * sizeof(int32_t));
     return l;
 }
 
@@ -304,17 +303,14 @@ vx_status make_cache_map_blocks(CUtensorMap *map, const void *ptr, int dim, int 
 
 // ------------------------------------------------------------------ shared launch pieces
 
-// sel_phys: NULL, or the physical page of each selection slot (written by the chained top-k)
 vx_status do_decode(const vx_geometry *g, const vx_page_table *t, const void *q, const void *k_cache,
-                    const void *v_cache, const int32_t *sel, const int32_t *sel_phys, int32_t k, float sm_scale,
-                    const Plan &p, const WsLayout &l, void *ws, void *out, float *lse, int32_t *err, cudaStream_t s,
-                    bool pdl) {
+                    const void *v_cache, const int32_t *sel, int32_t k, float sm_scale, const Plan &p,
+                    const WsLayout &l, void *ws, void *out, float *lse, int32_t *err, cudaStream_t s, bool pdl) {
     vx::DecodeArgs a{};
     a.page_ptr = t->page_ptr;
     a.page_indices = t->page_indices;
     a.seq_lens = t->seq_lens;
     a.sel = sel;
-    a.sel_phys = sel_phys;
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.o_part = reinterpret_cast<float *>(static_cast<char *>(ws) + l.o_part);
     a.ml_part = reinterpret_cast<float *>(static_cast<char *>(ws) + l.ml_part);
@@ -466,8 +462,7 @@ vx_status sparse_decode_compact(const vx_geometry *geo, const vx_page_table *tab
     if (!partials || !al16(partials)) return fail(VX_ERR_WORKSPACE, "partial buffer is NULL or not 16-byte aligned");
     if (partial_bytes < l.total)
         return fail(VX_ERR_WORKSPACE, "partial buffer of %zu bytes < %zu needed", partial_bytes, l.total);
-    return do_decode(geo, table, q, k_cache, v_cache, sel, nullptr, k, sm_scale, p, l, partials, out, lse, err, stream,
-                     false);
+    return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, partials, out, lse, err, stream, false);
 }
 
 }  // namespace vx
@@ -600,7 +595,7 @@ vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, c
     if (!ws || !al16(ws)) return fail(VX_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
     if (ws_bytes < decode_ws_bytes(l))
         return fail(VX_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, decode_ws_bytes(l));
-    return do_decode(geo, table, q, k_cache, v_cache, sel, nullptr, k, sm_scale, p, l, ws, out, lse, err,
+    return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, ws, out, lse, err,
                      static_cast<cudaStream_t>(stream), false);
 }
 
@@ -625,6 +620,8 @@ vx_status fused_step(const vx_geometry *geo, const vx_page_table *table, const v
     VX_TRY(check_ptr(lse, "lse", true));
     VX_TRY(check_ptr(scores_out, "scores_out", true));
     VX_TRY(check_ptr(sel_out, "sel_out", true));
+    const bool table_ready = (mode & VX_TABLE_READY) != 0;
+    mode &= ~VX_TABLE_READY;
     VX_TRY(check_k_mode(k, mode));
     VX_TRY(check_score_dims(geo, score_dims));
     if (err && !al4(err)) return fail(VX_ERR_INVALID_ARG, "err must be 4-byte aligned");
@@ -666,19 +663,15 @@ vx_status fused_step(const vx_geometry *geo, const vx_page_table *table, const v
         e = vx::launch_centroid(ca, vx::CEN_APPEND, s);
         if (e != cudaSuccess) return cuda_fail(e, "centroid append launch");
     }
-    // the scorer reads nothing before its dependency wait, so it may always launch early
-    e = vx::launch_score(score_args(geo, table, q, centroids, score_dims, scores, err), s, true);
+    // the scorer may always launch early: before its dependency wait it reads nothing, or
+    // (table_ready) only the page table and lengths
+    vx::ScoreArgs sa = score_args(geo, table, q, centroids, score_dims, scores, err);
+    sa.table_ready = table_ready ? 1 : 0;
+    e = vx::launch_score(sa, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "score launch");
-    // the top-k also writes each chosen page's physical id, so the decode's first copies wait on
-    // one load instead of two dependent ones
-    int32_t *sel_phys = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + l.sel_phys);
-    vx::TopkArgs ta = topk_args(geo, table, scores, k, seed, sel, err);
-    ta.page_ptr = table->page_ptr;
-    ta.page_indices = table->page_indices;
-    ta.sel_phys = sel_phys;
-    e = vx::launch_topk(ta, mode, s, true);
+    e = vx::launch_topk(topk_args(geo, table, scores, k, seed, sel, err), mode, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
-    return do_decode(geo, table, q, k_cache, v_cache, sel, sel_phys, k, sm_scale, p, l, ws, out, lse, err, s, true);
+    return do_decode(geo, table, q, k_cache, v_cache, sel, k, sm_scale, p, l, ws, out, lse, err, s, true);
 }
 
 }  // namespace

@@ -52,6 +52,7 @@ struct ScoreArgs {
     int32_t *err;
     int32_t B, Hq, Hkv, G, Dqk, P, max_pages, score_dims;
     int32_t qcap;             // requests whose summed query a block keeps in shared memory
+    int32_t table_ready;      // the table and lengths may be read before the dependency wait
     int64_t num_pool_pages;
 };
 
@@ -60,10 +61,6 @@ struct TopkArgs {
     const float *scores;
     int32_t *sel;
     int32_t *err;
-    // optional (sel_phys != NULL): the physical page of every chosen page, [B][Hkv][k], read
-    // from the table (page_ptr, page_indices) while the scores are still being computed
-    const int32_t *page_ptr, *page_indices;
-    int32_t *sel_phys;
     int32_t B, Hkv, P, max_pages, k, smem_keys;
     int32_t warp_max;  // exact rows of at most this many pages go to one warp (0: none)
     uint64_t seed;
@@ -71,7 +68,6 @@ struct TopkArgs {
 
 struct DecodeArgs {
     const int32_t *page_ptr, *page_indices, *seq_lens, *sel;
-    const int32_t *sel_phys;  // NULL, or the physical page of each selection slot (saves a lookup)
     const __nv_bfloat16 *q;
     float *o_part;   // [slots][G][Dv] unnormalised partial outputs
     float *ml_part;  // [slots][G][2]  (running max in log2 units, running sum)

@@ -138,8 +138,7 @@ constexpr int TOPK_WARP_MAX = 512;
 // private to the warp), then the ordered compaction over contiguous per-lane runs with warp
 // scans.  The chosen set is unique, so the result equals the block path's.
 static __device__ __noinline__ void warp_topk_small(const float *__restrict__ row, int n, int keff, int32_t *out, int k,
-                                                    uint32_t *skeys, int *hist, int32_t *out_phys,
-                                                    const int32_t *spages) {
+                                             uint32_t *skeys, int *hist) {
     const int lane = threadIdx.x & 31;
     {   // keys of the row (up to 16 loads per lane in flight)
         float v[TOPK_WARP_MAX / 32];
@@ -238,20 +237,14 @@ static __device__ __noinline__ void warp_topk_small(const float *__restrict__ ro
                 bool take = mk > prefix;
                 if (mk == prefix) take = eq_rank++ < remaining;
                 if (take) {
-                    if (pos < k) {
-                        out[pos] = j;
-                        if (out_phys) out_phys[pos] = spages[j];
-                    }
+                    if (pos < k) out[pos] = j;
                     ++pos;
                 }
             }
         }
     }
     const int sel_total = gt_total + min(eq_total, remaining);
-    for (int i = sel_total + lane; i < k; i += 32) {
-        out[i] = -1;
-        if (out_phys) out_phys[i] = -1;
-    }
+    for (int i = sel_total + lane; i < k; i += 32) out[i] = -1;
 }
 
 // Top-k of row (b, h) by the whole block (THREADS threads), written to a.sel.
@@ -260,10 +253,9 @@ static __device__ __noinline__ void warp_topk_small(const float *__restrict__ ro
 // dependent: the scores come from the previous kernel on the stream (wait for it before the
 // first score is read, and let the next kernel launch once the radix passes are done);
 // otherwise the caller has made them visible already.
-// spages: shared memory for a.smem_keys page ids (used when a.sel_phys is set).
 template <int ABITS, int THREADS>
 __device__ __forceinline__ void topk_row(const TopkArgs &a, int b, int h, TopkShared &sh, uint32_t *skeys,
-                                         int32_t *spages, bool dependent) {
+                                         bool dependent) {
     constexpr bool APPROX = ABITS > 0;
     constexpr int NCODES = APPROX ? (1 << ABITS) : 2;  // remap codes of the approximate mode
     static_assert(NCODES <= TOPK_HIST && (!APPROX || NCODES % THREADS == 0 || NCODES < THREADS),
@@ -279,26 +271,18 @@ __device__ __forceinline__ void topk_row(const TopkArgs &a, int b, int h, TopkSh
     }
     const int n = ceil_div(L, a.P);
     const int keff = min(a.k, n);
-    int32_t *out_phys = a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.k : nullptr;
-    const int32_t *prow = out_phys ? a.page_indices + a.page_ptr[b] : nullptr;  // the request's pages
     if (keff == n) {  // every page is chosen
-        for (int i = tid; i < a.k; i += THREADS) {
-            out[i] = i < n ? i : -1;
-            if (out_phys) out_phys[i] = i < n ? prow[i] : -1;
-        }
+        for (int i = tid; i < a.k; i += THREADS) out[i] = i < n ? i : -1;
         return;
     }
-    const bool in_smem = n <= a.smem_keys;
-    if (out_phys && in_smem)
-        for (int j = tid; j < n; j += THREADS) spages[j] = prow[j];
     // Everything above reads only inputs of the call, complete before this grid starts (it
     // runs in plain stream order or after the scorer, whose own dependency wait returned before
     // any of its blocks could end); the scores come from the previous kernel.
     if (dependent) pdl_wait();
+    const bool in_smem = n <= a.smem_keys;
     if constexpr (!APPROX && THREADS == 256) {
         if (n <= a.warp_max && in_smem) {  // uniform for the block: one warp does the row
-            __syncthreads();  // the page ids are staged
-            if (warp == 0) warp_topk_small(row, n, keff, out, a.k, skeys, sh.hist, out_phys, spages);
+            if (warp == 0) warp_topk_small(row, n, keff, out, a.k, skeys, sh.hist);
             return;
         }
     }
@@ -439,17 +423,11 @@ __device__ __forceinline__ void topk_row(const TopkArgs &a, int b, int h, TopkSh
             bool take = mk > prefix;
             if (mk == prefix) take = eq_rank++ < remaining;
             if (take) {
-                if (pos < a.k) {
-                    out[pos] = j;
-                    if (out_phys) out_phys[pos] = in_smem ? spages[j] : prow[j];
-                }
+                if (pos < a.k) out[pos] = j;
                 ++pos;
             }
         });
-        for (int i = sel_total + tid; i < a.k; i += THREADS) {
-            out[i] = -1;
-            if (out_phys) out_phys[i] = -1;
-        }
+        for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;
         return;
     }
     // approx: members of the boundary code are taken in cyclic page order from `offset`: first
@@ -498,18 +476,12 @@ __device__ __forceinline__ void topk_row(const TopkArgs &a, int b, int h, TopkSh
             bool take = mk > prefix;
             if (mk == prefix) take = (j < offset) ? lo_rank++ < take_lo : hi_rank++ < take_hi;
             if (take) {
-                if (pos < a.k) {
-                    out[pos] = j;
-                    if (out_phys) out_phys[pos] = in_smem ? spages[j] : prow[j];
-                }
+                if (pos < a.k) out[pos] = j;
                 ++pos;
             }
         });
     }
-    for (int i = sel_total + tid; i < a.k; i += THREADS) {
-        out[i] = -1;
-        if (out_phys) out_phys[i] = -1;
-    }
+    for (int i = sel_total + tid; i < a.k; i += THREADS) out[i] = -1;
 }
 
 }  // namespace vx

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libvx.so")
 VX_OK, VX_ERR_INVALID_ARG, VX_ERR_UNSUPPORTED, VX_ERR_WORKSPACE, VX_ERR_CUDA = range(5)
 VX_DATA_BAD_PAGE_ID, VX_DATA_BAD_SEQ_LEN, VX_DATA_BAD_SELECTION, VX_DATA_TIMEOUT = 1, 2, 4, 8
 NOALLOC_SCRATCH_BYTES = 16 << 20  # VX_NOALLOC_SCRATCH_BYTES of include/vx.h
+VX_TABLE_READY = 0x100  # mode flag of the chained steps: the table and lengths are not the previous kernel's output
 
 # every symbol include/vx.h declares
 EXPORTS = ["vx_centroid_update", "vx_score_pages", "vx_topk_pages", "vx_sparse_decode",

@@ -139,6 +139,20 @@ def test_appending_step_validation(L):
     assert L.vx_block_topk_decode_append(*args(FAKE, FAKE, 16)) == vx.VX_ERR_WORKSPACE
 
 
+def test_table_ready_flag_validation(L):
+    # VX_TABLE_READY is a flag of the chained steps' mode only; other bits are rejected
+    gp, tp = ctypes.byref(_geo()), ctypes.byref(_table())
+    f0 = ctypes.c_float(0.0)
+    step = lambda mode, ws_bytes: L.vx_block_topk_decode(gp, tp, FAKE, FAKE, FAKE, FAKE, 4, mode, 0, f0, 0, 8, FAKE,
+                                                         None, None, None, FAKE, ws_bytes, None, None)
+    assert step(vx.VX_TABLE_READY | 1, 16) == vx.VX_ERR_WORKSPACE  # the mode passed, the workspace did not
+    assert step(vx.VX_TABLE_READY << 1, 1 << 30) == vx.VX_ERR_INVALID_ARG
+    assert step(vx.VX_TABLE_READY | 4, 1 << 30) == vx.VX_ERR_INVALID_ARG
+    assert L.vx_topk_pages(gp, tp, FAKE, 4, vx.VX_TABLE_READY, 0, FAKE, None, None) == vx.VX_ERR_INVALID_ARG
+    hdr = open(os.path.join(ROOT, "include", "vx.h")).read()
+    assert f"#define VX_TABLE_READY {vx.VX_TABLE_READY:#x}" in hdr
+
+
 def test_persistent_step_validation(L):
     # vx_block_topk_decode_persistent refuses what it cannot run, before any launch
     tp = ctypes.byref(_table())

@@ -164,7 +164,8 @@ def test_fused_step_modes_match_separate_calls(name):
     for mode in (0, 1, 2, 3):
         for seed in (0, 77):
             err = err_word()
-            out, lse, s_f, sel_f = gpu_fused(w, cen, mode=mode, seed=seed, err=err)
+            flags = vx.VX_TABLE_READY if seed else 0  # the flag changes when reads start, not results
+            out, lse, s_f, sel_f = gpu_fused(w, cen, mode=mode | flags, seed=seed, err=err)
             assert np.array_equal(s_f.cpu().numpy(), s.cpu().numpy(), equal_nan=True)
             assert torch.equal(sel_f, gpu_topk(w, s, mode=mode, seed=seed))
             torch.cuda.synchronize()
@@ -173,11 +174,14 @@ def test_fused_step_modes_match_separate_calls(name):
                 break
 
 
+@pytest.mark.parametrize("flags", [0, vx.VX_TABLE_READY])
 @pytest.mark.parametrize("name", ["qwen_shape_small_batch", "mla_16heads", "g1_many_rows"])
-def test_fused_steps_on_a_stream_and_in_a_graph(name):
+def test_fused_steps_on_a_stream_and_in_a_graph(name, flags):
     """Back-to-back fused steps on a created stream (where the kernels' programmatic dependent
     launches take effect) and replayed from a CUDA graph give the default-stream result bit for
-    bit, with no device error (a bounded wait that ran out would set VX_DATA_TIMEOUT)."""
+    bit, with no device error (a bounded wait that ran out would set VX_DATA_TIMEOUT); with
+    VX_TABLE_READY too (each step's scorer then reads the table while the previous step's
+    merge runs)."""
     w = workload(name)
     cen = gpu_centroids(w)
     ref = gpu_fused(w, cen)
@@ -186,16 +190,16 @@ def test_fused_steps_on_a_stream_and_in_a_graph(name):
     err = err_word()
     bufs = [workspace(w) for _ in range(2)]
     with torch.cuda.stream(st):
-        runs = [gpu_fused(w, cen, err=err, ws=bufs[i % 2]) for i in range(6)]
+        runs = [gpu_fused(w, cen, err=err, ws=bufs[i % 2], mode=flags) for i in range(6)]
     torch.cuda.synchronize()
     outs = []
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(st):
-        gpu_fused(w, cen, err=err, ws=bufs[0])  # warm-up before capture
+        gpu_fused(w, cen, err=err, ws=bufs[0], mode=flags)  # warm-up before capture
         torch.cuda.synchronize()
         with torch.cuda.graph(g, stream=st):
             for i in range(4):
-                outs.append(gpu_fused(w, cen, err=err, ws=bufs[i % 2]))
+                outs.append(gpu_fused(w, cen, err=err, ws=bufs[i % 2], mode=flags))
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
@@ -276,9 +280,10 @@ def test_appending_step_equals_append_then_fused_call(mla):
             sc = torch.full((w.batch, spec.num_kv_heads, w.max_pages), float("nan"), device="cuda")
             sel = torch.empty((w.batch, spec.num_kv_heads, spec.k), dtype=torch.int32, device="cuda")
             v_new = None if w.step_v_new is None else w.step_v_new[s]  # MLA: the value is the latent key
-            if fused:
+            if fused:  # odd steps with VX_TABLE_READY (same results)
                 vx.vx_block_topk_decode_append(geo, tab, w.step_q[s], w.k_cache, w.v_cache, cen, w.step_k_new[s],
-                                               v_new, spec.k, out, ws, lse=lse, scores_out=sc, sel_out=sel, err=err)
+                                               v_new, spec.k, out, ws, lse=lse, scores_out=sc, sel_out=sel, err=err,
+                                               mode=vx.VX_TABLE_READY if s % 2 else 0)
             else:
                 vx.vx_centroid_update(geo, tab, w.k_cache, cen, v_cache=w.v_cache, k_new=w.step_k_new[s],
                                       v_new=v_new, err=err)
