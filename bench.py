@@ -518,12 +518,18 @@ def run_vx(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g_e, stream=stream):
             e2e_steps_on(chunk_e)
-    g_e.replay()
+    # warm-up: one untimed window of back-to-back replays, exactly like the timed one.  The
+    # first such window of a process runs about 1.7 ms slower in all (measured: 88.8 against
+    # 80.2 us per step over 200 steps, every later window 80.1-80.3), whatever the number of
+    # single synchronised replays before it; the device-only legs show no such step.
+    reps = max(1, e2e_steps // chunk_e)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g_e.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    reps = max(1, e2e_steps // chunk_e)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         ev0.record(stream)

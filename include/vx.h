@@ -164,9 +164,14 @@ vx_status vx_topk_pages(const vx_geometry *geo, const vx_page_table *table, cons
  * the page table.  For query head g of KV head h:
  *   out = sum_t softmax_t(sm_scale * q . K_t) V_t,  lse = log sum_t exp(sm_scale q . K_t)
  * over the valid tokens of the pages in sel[b][h] (entries < 0 skipped; entries must be
- * distinct).  Split-K: the selected tokens are cut into num_splits contiguous chunks
- * whose partial (o, max, sum) are merged with the log-sum-exp rule.
- *   sm_scale <= 0 means 1 / sqrt(head_dim_qk).  num_splits 0 = planned from the SM count.
+ * distinct).  Split-K: the selected tokens are cut into contiguous chunks whose partial
+ * (o, max, sum) are merged, in chunk order, with the log-sum-exp rule.
+ *   num_splits > 0: that many chunks of equal length (in 16-token tiles; MLA: pages).
+ *   num_splits 0: planned from the SM count.  MLA: one equal chunk per SM.  GQA: one equal
+ *   chunk per warp of a persistent grid over the first three quarters of the tiles, then
+ *   shorter equal chunks over the rest, each taken by whichever warp is free first.  The
+ *   chunks are fixed before launch, so results never depend on timing.
+ *   sm_scale <= 0 means 1 / sqrt(head_dim_qk).
  *   lse may be NULL.  A request with no attended token gets out = 0, lse = -inf.
  * ws: device workspace for the split partials; vx_workspace_size(geo, max_pages, k,
  * num_splits) bytes are always enough (that size also covers the fused call's scores
@@ -263,7 +268,7 @@ vx_status vx_block_topk_decode_persistent(const vx_geometry *geo, const vx_page_
  * split partials kept in one array of VX_NOALLOC_SCRATCH_BYTES that the library holds in
  * device memory, once per GPU, until the process exits.  It calls no cudaMalloc, cudaFree
  * or other allocating routine.
- *   - Limit: with W the split count after planning (num_splits, or the planned count for
+ *   - Limit: with W the chunk count after planning (num_splits, or vx_planned_splits for
  *     0, at most the number of tiles) and rows = batch * num_kv_heads, the partials take
  *     round_up_256((rows + W) * G * head_dim_v * 4) + (rows + W) * G * 2 * 4 bytes.  A
  *     problem that needs more than VX_NOALLOC_SCRATCH_BYTES is rejected with
@@ -297,7 +302,8 @@ vx_status vx_sparse_decode_noalloc(const vx_geometry *geo, const vx_page_table *
  */
 size_t vx_workspace_size(const vx_geometry *geo, int32_t max_pages, int32_t k, int32_t num_splits);
 
-/* Split count num_splits = 0 resolves to on the current device for this geometry. */
+/* Number of chunks the planned split (num_splits = 0) makes on the current device for this
+ * geometry.  Passing it as num_splits gives that many chunks of equal length instead. */
 int32_t vx_planned_splits(const vx_geometry *geo, int32_t max_pages, int32_t k);
 
 const char *vx_status_string(vx_status s);

@@ -7,14 +7,18 @@
 //
 // Work decomposition.  Every (request, KV head) row owns k selection slots; each slot
 // is a page of P tokens = P/16 tiles of 16 tokens.  The rows' tiles form one flat list
-// of T = rows * k * P/16 units, cut into W contiguous chunks of equal length; one warp
-// processes one chunk (a persistent grid: W = SMs * warps per block by default).  A
-// warp's chunk may end inside one row and continue in the next: for every row it
-// touches it writes one partial (unnormalised o, running max, running sum) to the
-// workspace at slot (row + chunk), an index that is unique because chunks are
-// contiguous.  The merge kernel combines a row's partials with the log-sum-exp rule.
-// The result therefore depends only on the selection and W, never on where the pages
-// live in the pool.
+// of T = rows * k * P/16 units, cut into contiguous pieces in unit order (piece_start):
+// Ws pieces of equal length over the first Us units, one per warp of a persistent grid,
+// then (planned split only) smaller equal pieces over the rest, which a warp takes as
+// soon as it is done with its previous piece, from a counter the step's scorer zeroed
+// (or round robin over the warps when there is no counter).  Warps that drew slow pages
+// then take fewer of the late pieces, so the launch ends closer to the mean warp's time.
+// A piece may end inside one row and continue in the next: for every row it touches it
+// writes one partial (unnormalised o, running max, running sum) to the workspace at slot
+// (row + piece), an index that is unique because pieces are contiguous and ordered.  The
+// merge kernel combines a row's partials in piece order with the log-sum-exp rule.  The
+// result therefore depends only on the selection and the piece layout, never on where
+// the pages live in the pool or which warp took which piece.
 //
 // Per warp: a ring of DEC_STAGES stages in shared memory, each holding one K tile and
 // one V tile (16 tokens x D bf16 each), each filled by one TMA tensor load (128-byte
@@ -34,6 +38,7 @@ namespace vx {
 struct TileMeta {
     int32_t row;
     int32_t nvalid;
+    int32_t piece;
 };
 
 __device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u, int64_t u_end) {
@@ -69,7 +74,9 @@ __device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u,
     return rs;
 }
 
-template <int D, int NT>
+// LATE: the split has late pieces (a.chunks > a.static_chunks); without them a warp's static
+// piece is all it does, and the piece bookkeeping compiles away.
+template <int D, int NT, bool LATE>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     k_decode_gqa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const DecodeArgs a) {
@@ -98,22 +105,33 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     }
     __syncwarp();
 
-    const int64_t c = (int64_t)blockIdx.x * DEC_WARPS + warp;
-    if (c >= a.chunks) return;
-    const int64_t u_begin = chunk_start(c, a.units, a.chunks);
-    const int64_t u_end = chunk_start(c + 1, a.units, a.chunks);
-    const int64_t row_first = u_begin / a.units_per_row;
-    const int64_t row_last = (u_end - 1) / a.units_per_row;
+    const int64_t wid = (int64_t)blockIdx.x * DEC_WARPS + warp;
+    if (wid >= a.static_chunks) return;
+    auto p_start = [&](int64_t c) -> int64_t {
+        return piece_start(c, a.units, a.static_units, a.static_chunks, a.chunks);
+    };
+    // the next piece this warp takes after its static one (warp-uniform): from the counter,
+    // or round robin over the warps
+    int64_t rr_next = a.static_chunks + wid;
+    auto next_piece = [&]() -> int64_t {
+        if constexpr (!LATE) return a.chunks;
+        if (a.piece_ctr) {
+            unsigned v = 0;
+            if (lane == 0) v = atomicAdd(a.piece_ctr, 1u);
+            return a.static_chunks + (int64_t)__shfl_sync(FULL, v, 0);
+        }
+        const int64_t c = rr_next;
+        rr_next += a.static_chunks;
+        return c;
+    };
 
     // ---- per-row state
     uint32_t qf[NT][MT][2];
     float acc[NT][MT][4];
     float m_run[NT][2], l_run[NT][2];
-    int64_t cur_row = -1;
-    int64_t flushed_to = row_first - 1;  // rows <= flushed_to have their partial written
 
-    // partial of row `r` (at least one tile attended) for this chunk: slot r + c
-    auto write_partial = [&](int64_t r) {
+    // partial of row `r` (at least one tile attended) for piece `c`: slot r + c
+    auto write_partial = [&](int64_t r, int64_t c) {
         const int64_t slot = r + c;
         float lt[NT][2];
 #pragma unroll
@@ -150,12 +168,17 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
                 }
         }
     };
-    auto empty_partial = [&](int64_t r) {
-        if (lane < a.G) {
-            float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
-            ml[0] = -INFINITY;
-            ml[1] = 0.f;
-        }
+    // every row that piece c touches starts with an empty partial (max -inf, sum 0); rows
+    // with attended tiles get theirs overwritten later by this same warp
+    auto empty_piece = [&](int64_t c) {
+        const int64_t u0 = p_start(c), u1 = p_start(c + 1);
+        for (int64_t r = u0 / a.units_per_row; r <= (u1 - 1) / a.units_per_row; ++r)
+            if (lane < a.G) {
+                float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
+                ml[0] = -INFINITY;
+                ml[1] = 0.f;
+            }
+        __syncwarp();
     };
     auto start_row = [&](int64_t r) {
         const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);
@@ -190,24 +213,40 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     // input of the call, complete before this grid starts (the grid runs either in plain
     // stream order or after the top-k kernel, which itself starts after the scorer ends).
     // Only the selection is written by the previous kernel.
-    start_row(row_first);
-    cur_row = row_first;
+    // The static piece's empty partials are written before the wait as well: the workspace is
+    // not touched by the previous kernel (the top-k, or nothing in plain stream order).
+    int64_t fc = wid, batch = p_start(wid), f_end = p_start(wid + 1);
+    int64_t cur_row = batch / a.units_per_row, cur_pc = wid;  // (row, piece) being accumulated
+    start_row(cur_row);
+    empty_piece(fc);
     pdl_wait();
 
-    // ---- pipeline
-    int64_t batch = u_begin;
-    Resolved rs = resolve_unit(a, batch + lane, u_end);
+    // ---- pipeline: the filler resolves and issues the units of piece fc in [batch, f_end),
+    // then takes the next piece; the consumer attends tile after tile
+    bool fill_done = false;
+    Resolved rs = resolve_unit(a, batch + lane, f_end);
     uint32_t pending = __ballot_sync(FULL, rs.valid);
     uint32_t issued = 0, consumed = 0;
     bool failed = false;
 
     for (;;) {
-        // issue loads until the ring is full or the chunk is exhausted
+        // issue loads until the ring is full or no piece is left
         while (!failed && issued - consumed < DEC_STAGES) {
             if (pending == 0) {
                 batch += 32;
-                if (batch >= u_end) break;
-                rs = resolve_unit(a, batch + lane, u_end);
+                if (batch >= f_end) {
+                    if (fill_done) break;
+                    const int64_t c = next_piece();
+                    if (c >= a.chunks) {
+                        fill_done = true;
+                        break;
+                    }
+                    fc = c;
+                    batch = p_start(c);
+                    f_end = p_start(c + 1);
+                    empty_piece(c);
+                }
+                rs = resolve_unit(a, batch + lane, f_end);
                 pending = __ballot_sync(FULL, rs.valid);
                 continue;
             }
@@ -221,6 +260,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             if (lane == 0) {
                 meta[st].row = row;
                 meta[st].nvalid = nv;
+                if constexpr (LATE) meta[st].piece = static_cast<int32_t>(fc);
                 const uint32_t bar = bar0 + 8u * st;
                 const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
                 // no proxy fence: this stage's earlier shared-memory reads have completed,
@@ -232,35 +272,38 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             __syncwarp();
             ++issued;
         }
-        // next tile (or the end of the chunk: row = row_last + 1)
-        int64_t row = row_last + 1;
+        // next tile, or the end (row -1)
+        int64_t row = -1, pc = -1;
         int nvalid = 0;
         int st = 0;
         if (!failed && consumed != issued) {
             st = static_cast<int>(consumed % DEC_STAGES);
             if (!__all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
-                // a load did not arrive in time: report, let every issued load land and
-                // finish the remaining rows as empty
+                // a load did not arrive in time: report, let every issued load land, drop the
+                // partial in progress (its slot keeps its empty partial) and give every piece
+                // this warp would still have taken its empty partials
                 if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
                 for (uint32_t i = consumed; i < issued; ++i)
                     (void)mbar_wait_bounded(bar0 + 8u * (i % DEC_STAGES), (i / DEC_STAGES) & 1u);
                 failed = true;
                 cur_row = -1;
+                while (!fill_done) {
+                    const int64_t c = next_piece();
+                    if (c >= a.chunks) fill_done = true;
+                    else empty_piece(c);
+                }
             } else {
                 row = meta[st].row;
                 nvalid = meta[st].nvalid;
+                pc = LATE ? meta[st].piece : cur_pc;
             }
         }
-        if (row != cur_row) {
-            if (cur_row >= 0) {
-                write_partial(cur_row);
-                flushed_to = cur_row;
-            }
-            for (int64_t r = flushed_to + 1; r < row; ++r) empty_partial(r);
-            flushed_to = row - 1;
-            if (row > row_last) break;
+        if (row != cur_row || (LATE && pc != cur_pc)) {
+            if (cur_row >= 0) write_partial(cur_row, cur_pc);
+            if (row < 0) break;
             start_row(row);
             cur_row = row;
+            cur_pc = pc;
         }
 
         const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
@@ -297,8 +340,8 @@ __global__ void __launch_bounds__(256) k_merge(const DecodeArgs a) {
     const int64_t rg = item / NSLICE;
     const int64_t r = rg / a.G;
     const int g = static_cast<int>(rg % a.G);
-    const int64_t c_lo = chunk_of(r * a.units_per_row, a.units, a.chunks);
-    const int64_t c_hi = chunk_of((r + 1) * a.units_per_row - 1, a.units, a.chunks);
+    const int64_t c_lo = piece_of(r * a.units_per_row, a.units, a.static_units, a.static_chunks, a.chunks);
+    const int64_t c_hi = piece_of((r + 1) * a.units_per_row - 1, a.units, a.static_units, a.static_chunks, a.chunks);
     const int np = static_cast<int>(c_hi - c_lo + 1);
     const float *ml0 = a.ml_part + ((r + c_lo) * a.G + g) * 2;                               // partial i at + i*G*2
     const float *o0 = a.o_part + ((r + c_lo) * a.G + g) * DV + slice * SLICE + lane * PER;   // partial i at + i*G*DV
@@ -376,9 +419,10 @@ static cudaError_t launch_gqa_dn(const DecodeArgs &a, const CUtensorMap &tmK, co
                                  int grid, cudaStream_t s, bool pdl) {
     constexpr int STAGE_BYTES = 2 * DEC_TILE * D * 2;
     const size_t smem = 1024 + (size_t)DEC_WARPS * DEC_STAGES * (STAGE_BYTES + 8 + sizeof(TileMeta));
-    auto kern = k_decode_gqa<D, NT>;
-    static std::atomic<unsigned long long> done;
-    cudaError_t e = ensure_smem_limit(kern, (int)smem, done);
+    const bool late = a.chunks > a.static_chunks;
+    auto kern = late ? k_decode_gqa<D, NT, true> : k_decode_gqa<D, NT, false>;
+    static std::atomic<unsigned long long> done[2];
+    cudaError_t e = ensure_smem_limit(kern, (int)smem, done[late ? 1 : 0]);
     if (e != cudaSuccess) return e;
     return launch_k(kern, dim3(grid), dim3(DEC_WARPS * 32), smem, s, pdl, tmK, tmV, a);
 }
@@ -402,8 +446,12 @@ static cudaError_t launch_merge_dv(const DecodeArgs &a, cudaStream_t s, bool pdl
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)a.B * a.Hkv;
     const int64_t wide_items = rows * a.G * (DV / (32 * PW));
-    // partials of the row with the most: the chunks it spans
-    const int64_t np_max = (a.units_per_row * a.chunks + a.units - 1) / a.units + 1;
+    // partials of the row with the most: the pieces it spans in each region of the split
+    int64_t np_max = (a.units_per_row * a.static_chunks + a.static_units - 1) / a.static_units + 1;
+    if (a.chunks > a.static_chunks) {
+        const int64_t ud = a.units - a.static_units, wd = a.chunks - a.static_chunks;
+        np_max += (a.units_per_row * wd + ud - 1) / ud + 1;
+    }
     // the narrow shapes keep 24 (16-partial groups) or 16 (32-partial groups) warps resident
     // per SM; more warps than that would run in several waves
     const int64_t narrow_items = rows * a.G * (DV / 32);

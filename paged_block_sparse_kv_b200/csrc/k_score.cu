@@ -162,6 +162,8 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
     }
     if (a.table_ready) pdl_wait();
     if (bad_len && blockIdx.x == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
+    // the decode kernel later in the same step counts its late pieces from this word
+    if (a.zero_word && blockIdx.x == 0 && threadIdx.x == 0) *a.zero_word = 0u;
 
     // ---- group-summed queries of the block's first requests, computed once per block: each
     // thread sums one (request, KV head, 8-dim chunk) over the group's heads in head order

@@ -26,6 +26,9 @@ constexpr int APPROX_BITS_COARSE = 8;    // approximate top-k, mode 3: 256 codes
 constexpr int DEC_WARPS = 8;             // GQA decode: worker warps per block
 constexpr int DEC_STAGES = 3;            // GQA decode: 16-token tiles in flight per warp
 constexpr int DEC_TILE = 16;             // GQA decode: tokens per tile (one mma M or K step)
+constexpr int DEC_DYN_PCT = 25;          // GQA decode, planned split: % of tiles handed out late
+constexpr int DEC_DYN_DIV = 8;           // ... in pieces of 1 / DEC_DYN_DIV of a warp's share of tiles
+constexpr int DEC_DYN_MIN_PIECE = 8;     // ... only when such a piece has at least this many tiles
 constexpr int MLA_MIN_PAGE = 32;         // MLA decode: pages of 32 or 64 tokens
 constexpr int MLA_TILE_ROWS = 64;        // MLA decode: tokens per tile (a page of up to 64 tokens)
 
@@ -53,6 +56,7 @@ struct ScoreArgs {
     int32_t B, Hq, Hkv, G, Dqk, P, max_pages, score_dims;
     int32_t qcap;             // requests whose summed query a block keeps in shared memory
     int32_t table_ready;      // the table and lengths may be read before the dependency wait
+    uint32_t *zero_word;      // NULL, or a word block 0 sets to zero after the dependency wait
     int64_t num_pool_pages;
 };
 
@@ -79,6 +83,12 @@ struct DecodeArgs {
     int64_t num_pool_pages;
     int64_t units;            // rows * k * tiles_per_page
     int64_t units_per_row;    // k * tiles_per_page
+    // pieces (`chunks` in all): the first static_chunks split units [0, static_units) evenly,
+    // the rest split [static_units, units) evenly (see piece_start)
+    int64_t static_units;
+    int32_t static_chunks;
+    uint32_t *piece_ctr;      // NULL: warp w takes pieces w, static_chunks + w, + 2 static_chunks ...;
+                              // else pieces past the first static_chunks come from this counter (zero at launch)
     int32_t chunks;           // split count W
     float scale_log2;         // sm_scale * log2(e)
 };
@@ -198,6 +208,17 @@ __host__ __device__ __forceinline__ int64_t chunk_start(int64_t c, int64_t T, in
 // the chunk holding unit u
 __host__ __device__ __forceinline__ int64_t chunk_of(int64_t u, int64_t T, int64_t W) {
     return ((u + 1) * W - 1) / T;
+}
+
+// Pieces of the decode split: pieces 0 .. Ws-1 cut units [0, Us) into Ws equal chunks, pieces
+// Ws .. W-1 cut [Us, T) into W - Ws equal chunks (Us == T and Ws == W: the plain even split).
+// Every piece holds at least one unit; pieces are contiguous and in unit order, so slot
+// (row + piece) is unique for every (row, piece) pair that shares a unit.
+__host__ __device__ __forceinline__ int64_t piece_start(int64_t c, int64_t T, int64_t Us, int64_t Ws, int64_t W) {
+    return c <= Ws ? chunk_start(c, Us, Ws) : Us + chunk_start(c - Ws, T - Us, W - Ws);
+}
+__host__ __device__ __forceinline__ int64_t piece_of(int64_t u, int64_t T, int64_t Us, int64_t Ws, int64_t W) {
+    return u < Us ? chunk_of(u, Us, Ws) : Ws + chunk_of(u - Us, T - Us, W - Ws);
 }
 
 }  // namespace vx

@@ -26,6 +26,10 @@ CASES = {
                                           ctx=("list", [40, 90]), k=20), 15),
     "qwen_shape_small_batch": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=8, head_dim_qk=128,
                                                  page_size=16, ctx=("uniform", 4096, 9000), k=128, n_planted=8), 16),
+    # 81920 tiles, about 69 per warp on 148 SMs: enough that the planned split hands a quarter
+    # of them out late, in pieces, from a counter; short contexts leave -1 selection slots
+    "late_pieces_b64": (synth.custom_spec(batch=64, num_q_heads=16, num_kv_heads=8, head_dim_qk=128, page_size=16,
+                                          ctx=("uniform", 1500, 5000), k=160), 20),
     "mla_16heads": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
                                       page_size=64, mla_shared_kv=True, ctx=("list", [700, 2000, 64]), k=6), 17),
     "mla_5heads_ragged": (synth.custom_spec(batch=2, num_q_heads=5, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
@@ -154,7 +158,8 @@ def test_approx_topk_bit_exact_on_gpu_scores(name):
     assert recall(sel.cpu().numpy(), exact) > 0.5
 
 
-@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "mla_16heads", "g16_d64_page64", "edges_1tok_fullpage_ragged"])
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "mla_16heads", "g16_d64_page64", "edges_1tok_fullpage_ragged",
+                                  "late_pieces_b64"])
 def test_fused_step_modes_match_separate_calls(name):
     """The fused step in every top-k mode gives the separate calls' scores and selection bit for
     bit (the chained kernels run with programmatic dependent launch)."""
@@ -168,6 +173,10 @@ def test_fused_step_modes_match_separate_calls(name):
             out, lse, s_f, sel_f = gpu_fused(w, cen, mode=mode | flags, seed=seed, err=err)
             assert np.array_equal(s_f.cpu().numpy(), s.cpu().numpy(), equal_nan=True)
             assert torch.equal(sel_f, gpu_topk(w, s, mode=mode, seed=seed))
+            # the planned split hands its late pieces to whichever warp is free in the fused step
+            # and round robin in the separate call: same pieces, same partial slots, same bits
+            out_d, lse_d = gpu_decode(w, sel_f)
+            assert torch.equal(out.view(torch.int16), out_d.view(torch.int16)) and torch.equal(lse, lse_d)
             torch.cuda.synchronize()
             assert int(err.item()) == 0
             if mode == 0:
@@ -175,7 +184,7 @@ def test_fused_step_modes_match_separate_calls(name):
 
 
 @pytest.mark.parametrize("flags", [0, vx.VX_TABLE_READY])
-@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "mla_16heads", "g1_many_rows"])
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "mla_16heads", "g1_many_rows", "late_pieces_b64"])
 def test_fused_steps_on_a_stream_and_in_a_graph(name, flags):
     """Back-to-back fused steps on a created stream (where the kernels' programmatic dependent
     launches take effect) and replayed from a CUDA graph give the default-stream result bit for
@@ -464,3 +473,11 @@ def test_empty_selection_rows(name):
     check_attention(out, lse, o_orc, l_orc)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
+
+
+def test_late_pieces_case_has_late_pieces():
+    """The planned split of late_pieces_b64 has late pieces on this GPU (more chunks than warps),
+    so the parity cases that use it cover them."""
+    w = workload("late_pieces_b64")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert vx.vx_planned_splits(geometry(w), w.max_pages, w.spec.k) > sms * 8
