@@ -35,10 +35,16 @@
 
 namespace vx {
 
+template <bool LATE>
 struct TileMeta {
     int32_t row;
     int32_t nvalid;
-    int32_t piece;
+    int32_t piece;  // the piece the tile belongs to (split with late pieces)
+};
+template <>
+struct TileMeta<false> {
+    int32_t row;
+    int32_t nvalid;
 };
 
 __device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u, int64_t u_end) {
@@ -74,8 +80,9 @@ __device__ __forceinline__ Resolved resolve_unit(const DecodeArgs &a, int64_t u,
     return rs;
 }
 
-// LATE: the split has late pieces (a.chunks > a.static_chunks); without them a warp's static
-// piece is all it does, and the piece bookkeeping compiles away.
+// LATE: the split has late pieces (a.chunks > a.static_chunks).  Without them a warp's static
+// piece is all it does and the kernel runs the plain one-chunk-per-warp loop (the piece
+// bookkeeping cost the headline and long-context steps 0.4-2 us when compiled in).
 template <int D, int NT, bool LATE>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     k_decode_gqa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -93,7 +100,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     const int g4 = lane >> 2, q4 = lane & 3;
     const uint32_t stage0 = base + (uint32_t)(warp * DEC_STAGES) * STAGE_BYTES;
     const uint32_t bar0 = base + (uint32_t)(DEC_WARPS * DEC_STAGES) * STAGE_BYTES + (uint32_t)(warp * DEC_STAGES) * 8u;
-    TileMeta *meta = reinterpret_cast<TileMeta *>(smem_raw + (base - raw) + DEC_WARPS * DEC_STAGES * STAGE_BYTES +
+    TileMeta<LATE> *meta = reinterpret_cast<TileMeta<LATE> *>(smem_raw + (base - raw) + DEC_WARPS * DEC_STAGES * STAGE_BYTES +
                                                   DEC_WARPS * DEC_STAGES * 8) +
                      warp * DEC_STAGES;
 
@@ -107,24 +114,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 
     const int64_t wid = (int64_t)blockIdx.x * DEC_WARPS + warp;
     if (wid >= a.static_chunks) return;
-    auto p_start = [&](int64_t c) -> int64_t {
-        return piece_start(c, a.units, a.static_units, a.static_chunks, a.chunks);
-    };
-    // the next piece this warp takes after its static one (warp-uniform): from the counter,
-    // or round robin over the warps
-    int64_t rr_next = a.static_chunks + wid;
-    auto next_piece = [&]() -> int64_t {
-        if constexpr (!LATE) return a.chunks;
-        if (a.piece_ctr) {
-            unsigned v = 0;
-            if (lane == 0) v = atomicAdd(a.piece_ctr, 1u);
-            return a.static_chunks + (int64_t)__shfl_sync(FULL, v, 0);
-        }
-        const int64_t c = rr_next;
-        rr_next += a.static_chunks;
-        return c;
-    };
-
     // ---- per-row state
     uint32_t qf[NT][MT][2];
     float acc[NT][MT][4];
@@ -170,16 +159,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     };
     // every row that piece c touches starts with an empty partial (max -inf, sum 0); rows
     // with attended tiles get theirs overwritten later by this same warp
-    auto empty_piece = [&](int64_t c) {
-        const int64_t u0 = p_start(c), u1 = p_start(c + 1);
-        for (int64_t r = u0 / a.units_per_row; r <= (u1 - 1) / a.units_per_row; ++r)
-            if (lane < a.G) {
-                float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
-                ml[0] = -INFINITY;
-                ml[1] = 0.f;
-            }
-        __syncwarp();
-    };
     auto start_row = [&](int64_t r) {
         const int b = static_cast<int>(r / a.Hkv), h = static_cast<int>(r % a.Hkv);
         const __nv_bfloat16 *qb = a.q + ((size_t)b * a.Hq + (size_t)h * a.G) * D;
@@ -209,107 +188,234 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         }
     };
 
-    // The first row's query is read before waiting on the previous kernel: the query is an
-    // input of the call, complete before this grid starts (the grid runs either in plain
-    // stream order or after the top-k kernel, which itself starts after the scorer ends).
-    // Only the selection is written by the previous kernel.
-    // The static piece's empty partials are written before the wait as well: the workspace is
-    // not touched by the previous kernel (the top-k, or nothing in plain stream order).
-    int64_t fc = wid, batch = p_start(wid), f_end = p_start(wid + 1);
-    int64_t cur_row = batch / a.units_per_row, cur_pc = wid;  // (row, piece) being accumulated
-    start_row(cur_row);
-    empty_piece(fc);
-    pdl_wait();
+    if constexpr (!LATE) {
+        // one static piece per warp: the even split
+        const int64_t c = wid;
+        const int64_t u_begin = chunk_start(c, a.units, a.chunks);
+        const int64_t u_end = chunk_start(c + 1, a.units, a.chunks);
+        const int64_t row_first = u_begin / a.units_per_row;
+        const int64_t row_last = (u_end - 1) / a.units_per_row;
+        int64_t cur_row = -1;
+        int64_t flushed_to = row_first - 1;  // rows <= flushed_to have their partial written
+        auto empty_partial = [&](int64_t r) {
+            if (lane < a.G) {
+                float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
+                ml[0] = -INFINITY;
+                ml[1] = 0.f;
+            }
+        };
+        // The first row's query is read before waiting on the previous kernel: the query is an
+        // input of the call, complete before this grid starts (the grid runs either in plain
+        // stream order or after the top-k kernel, which itself starts after the scorer ends).
+        // Only the selection is written by the previous kernel.
+        start_row(row_first);
+        cur_row = row_first;
+        pdl_wait();
 
-    // ---- pipeline: the filler resolves and issues the units of piece fc in [batch, f_end),
-    // then takes the next piece; the consumer attends tile after tile
-    bool fill_done = false;
-    Resolved rs = resolve_unit(a, batch + lane, f_end);
-    uint32_t pending = __ballot_sync(FULL, rs.valid);
-    uint32_t issued = 0, consumed = 0;
-    bool failed = false;
+        // ---- pipeline
+        int64_t batch = u_begin;
+        Resolved rs = resolve_unit(a, batch + lane, u_end);
+        uint32_t pending = __ballot_sync(FULL, rs.valid);
+        uint32_t issued = 0, consumed = 0;
+        bool failed = false;
 
-    for (;;) {
-        // issue loads until the ring is full or no piece is left
-        while (!failed && issued - consumed < DEC_STAGES) {
-            if (pending == 0) {
-                batch += 32;
-                if (batch >= f_end) {
-                    if (fill_done) break;
-                    const int64_t c = next_piece();
-                    if (c >= a.chunks) {
-                        fill_done = true;
-                        break;
-                    }
-                    fc = c;
-                    batch = p_start(c);
-                    f_end = p_start(c + 1);
-                    empty_piece(c);
+        for (;;) {
+            // issue loads until the ring is full or the chunk is exhausted
+            while (!failed && issued - consumed < DEC_STAGES) {
+                if (pending == 0) {
+                    batch += 32;
+                    if (batch >= u_end) break;
+                    rs = resolve_unit(a, batch + lane, u_end);
+                    pending = __ballot_sync(FULL, rs.valid);
+                    continue;
                 }
-                rs = resolve_unit(a, batch + lane, f_end);
-                pending = __ballot_sync(FULL, rs.valid);
-                continue;
+                const int src = __ffs(pending) - 1;
+                pending &= pending - 1;
+                const int32_t row = __shfl_sync(FULL, rs.row, src);
+                const int32_t z = __shfl_sync(FULL, rs.z, src);
+                const int32_t y = __shfl_sync(FULL, rs.y, src);
+                const int32_t nv = __shfl_sync(FULL, rs.nvalid, src);
+                const int st = static_cast<int>(issued % DEC_STAGES);
+                if (lane == 0) {
+                    meta[st].row = row;
+                    meta[st].nvalid = nv;
+                    const uint32_t bar = bar0 + 8u * st;
+                    const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
+                    // no proxy fence: this stage's earlier shared-memory reads have completed,
+                    // their values were consumed before the __syncwarp that released the stage
+                    mbar_arrive_expect_tx(bar, STAGE_BYTES);
+                    tma_load_4d(sK, &tmK, 0, y, 0, z, bar);
+                    tma_load_4d(sK + TILE_BYTES, &tmV, 0, y, 0, z, bar);
+                }
+                __syncwarp();
+                ++issued;
             }
-            const int src = __ffs(pending) - 1;
-            pending &= pending - 1;
-            const int32_t row = __shfl_sync(FULL, rs.row, src);
-            const int32_t z = __shfl_sync(FULL, rs.z, src);
-            const int32_t y = __shfl_sync(FULL, rs.y, src);
-            const int32_t nv = __shfl_sync(FULL, rs.nvalid, src);
-            const int st = static_cast<int>(issued % DEC_STAGES);
-            if (lane == 0) {
-                meta[st].row = row;
-                meta[st].nvalid = nv;
-                if constexpr (LATE) meta[st].piece = static_cast<int32_t>(fc);
-                const uint32_t bar = bar0 + 8u * st;
-                const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
-                // no proxy fence: this stage's earlier shared-memory reads have completed,
-                // their values were consumed before the __syncwarp that released the stage
-                mbar_arrive_expect_tx(bar, STAGE_BYTES);
-                tma_load_4d(sK, &tmK, 0, y, 0, z, bar);
-                tma_load_4d(sK + TILE_BYTES, &tmV, 0, y, 0, z, bar);
+            // next tile (or the end of the chunk: row = row_last + 1)
+            int64_t row = row_last + 1;
+            int nvalid = 0;
+            int st = 0;
+            if (!failed && consumed != issued) {
+                st = static_cast<int>(consumed % DEC_STAGES);
+                if (!__all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
+                    // a load did not arrive in time: report, let every issued load land and
+                    // finish the remaining rows as empty
+                    if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
+                    for (uint32_t i = consumed; i < issued; ++i)
+                        (void)mbar_wait_bounded(bar0 + 8u * (i % DEC_STAGES), (i / DEC_STAGES) & 1u);
+                    failed = true;
+                    cur_row = -1;
+                } else {
+                    row = meta[st].row;
+                    nvalid = meta[st].nvalid;
+                }
             }
+            if (row != cur_row) {
+                if (cur_row >= 0) {
+                    write_partial(cur_row, c);
+                    flushed_to = cur_row;
+                }
+                for (int64_t r = flushed_to + 1; r < row; ++r) empty_partial(r);
+                flushed_to = row - 1;
+                if (row > row_last) break;
+                start_row(row);
+                cur_row = row;
+            }
+
+            const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
+            attend_tile<D, NT>(sK, sK + TILE_BYTES, nvalid, a.scale_log2, qf, acc, m_run, l_run, lane);
+            __syncwarp();  // every lane is done with this stage before it is refilled
+            ++consumed;
+        }
+    } else {
+        auto p_start = [&](int64_t c) -> int64_t {
+            return piece_start(c, a.units, a.static_units, a.static_chunks, a.chunks);
+        };
+        // the next piece this warp takes after its static one (warp-uniform): from the counter,
+        // or round robin over the warps
+        int64_t rr_next = a.static_chunks + wid;
+        auto next_piece = [&]() -> int64_t {
+            if (a.piece_ctr) {
+                unsigned v = 0;
+                if (lane == 0) v = atomicAdd(a.piece_ctr, 1u);
+                return a.static_chunks + (int64_t)__shfl_sync(FULL, v, 0);
+            }
+            const int64_t c = rr_next;
+            rr_next += a.static_chunks;
+            return c;
+        };
+
+        auto empty_piece = [&](int64_t c) {
+            const int64_t u0 = p_start(c), u1 = p_start(c + 1);
+            for (int64_t r = u0 / a.units_per_row; r <= (u1 - 1) / a.units_per_row; ++r)
+                if (lane < a.G) {
+                    float *ml = a.ml_part + ((r + c) * a.G + lane) * 2;
+                    ml[0] = -INFINITY;
+                    ml[1] = 0.f;
+                }
             __syncwarp();
-            ++issued;
-        }
-        // next tile, or the end (row -1)
-        int64_t row = -1, pc = -1;
-        int nvalid = 0;
-        int st = 0;
-        if (!failed && consumed != issued) {
-            st = static_cast<int>(consumed % DEC_STAGES);
-            if (!__all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
-                // a load did not arrive in time: report, let every issued load land, drop the
-                // partial in progress (its slot keeps its empty partial) and give every piece
-                // this warp would still have taken its empty partials
-                if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
-                for (uint32_t i = consumed; i < issued; ++i)
-                    (void)mbar_wait_bounded(bar0 + 8u * (i % DEC_STAGES), (i / DEC_STAGES) & 1u);
-                failed = true;
-                cur_row = -1;
-                while (!fill_done) {
-                    const int64_t c = next_piece();
-                    if (c >= a.chunks) fill_done = true;
-                    else empty_piece(c);
-                }
-            } else {
-                row = meta[st].row;
-                nvalid = meta[st].nvalid;
-                pc = LATE ? meta[st].piece : cur_pc;
-            }
-        }
-        if (row != cur_row || (LATE && pc != cur_pc)) {
-            if (cur_row >= 0) write_partial(cur_row, cur_pc);
-            if (row < 0) break;
-            start_row(row);
-            cur_row = row;
-            cur_pc = pc;
-        }
+        };
+        // The first row's query is read before waiting on the previous kernel: the query is an
+        // input of the call, complete before this grid starts (the grid runs either in plain
+        // stream order or after the top-k kernel, which itself starts after the scorer ends).
+        // Only the selection is written by the previous kernel.
+        // The static piece's empty partials are written before the wait as well: the workspace is
+        // not touched by the previous kernel (the top-k, or nothing in plain stream order).
+        int64_t fc = wid, batch = p_start(wid), f_end = p_start(wid + 1);
+        int64_t cur_row = batch / a.units_per_row, cur_pc = wid;  // (row, piece) being accumulated
+        start_row(cur_row);
+        empty_piece(fc);
+        pdl_wait();
 
-        const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
-        attend_tile<D, NT>(sK, sK + TILE_BYTES, nvalid, a.scale_log2, qf, acc, m_run, l_run, lane);
-        __syncwarp();  // every lane is done with this stage before it is refilled
-        ++consumed;
+        // ---- pipeline: the filler resolves and issues the units of piece fc in [batch, f_end),
+        // then takes the next piece; the consumer attends tile after tile
+        bool fill_done = false;
+        Resolved rs = resolve_unit(a, batch + lane, f_end);
+        uint32_t pending = __ballot_sync(FULL, rs.valid);
+        uint32_t issued = 0, consumed = 0;
+        bool failed = false;
+
+        for (;;) {
+            // issue loads until the ring is full or no piece is left
+            while (!failed && issued - consumed < DEC_STAGES) {
+                if (pending == 0) {
+                    batch += 32;
+                    if (batch >= f_end) {
+                        if (fill_done) break;
+                        const int64_t c = next_piece();
+                        if (c >= a.chunks) {
+                            fill_done = true;
+                            break;
+                        }
+                        fc = c;
+                        batch = p_start(c);
+                        f_end = p_start(c + 1);
+                        empty_piece(c);
+                    }
+                    rs = resolve_unit(a, batch + lane, f_end);
+                    pending = __ballot_sync(FULL, rs.valid);
+                    continue;
+                }
+                const int src = __ffs(pending) - 1;
+                pending &= pending - 1;
+                const int32_t row = __shfl_sync(FULL, rs.row, src);
+                const int32_t z = __shfl_sync(FULL, rs.z, src);
+                const int32_t y = __shfl_sync(FULL, rs.y, src);
+                const int32_t nv = __shfl_sync(FULL, rs.nvalid, src);
+                const int st = static_cast<int>(issued % DEC_STAGES);
+                if (lane == 0) {
+                    meta[st].row = row;
+                    meta[st].nvalid = nv;
+                    meta[st].piece = static_cast<int32_t>(fc);
+                    const uint32_t bar = bar0 + 8u * st;
+                    const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
+                    // no proxy fence: this stage's earlier shared-memory reads have completed,
+                    // their values were consumed before the __syncwarp that released the stage
+                    mbar_arrive_expect_tx(bar, STAGE_BYTES);
+                    tma_load_4d(sK, &tmK, 0, y, 0, z, bar);
+                    tma_load_4d(sK + TILE_BYTES, &tmV, 0, y, 0, z, bar);
+                }
+                __syncwarp();
+                ++issued;
+            }
+            // next tile, or the end (row -1)
+            int64_t row = -1, pc = -1;
+            int nvalid = 0;
+            int st = 0;
+            if (!failed && consumed != issued) {
+                st = static_cast<int>(consumed % DEC_STAGES);
+                if (!__all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
+                    // a load did not arrive in time: report, let every issued load land, drop the
+                    // partial in progress (its slot keeps its empty partial) and give every piece
+                    // this warp would still have taken its empty partials
+                    if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
+                    for (uint32_t i = consumed; i < issued; ++i)
+                        (void)mbar_wait_bounded(bar0 + 8u * (i % DEC_STAGES), (i / DEC_STAGES) & 1u);
+                    failed = true;
+                    cur_row = -1;
+                    while (!fill_done) {
+                        const int64_t c = next_piece();
+                        if (c >= a.chunks) fill_done = true;
+                        else empty_piece(c);
+                    }
+                } else {
+                    row = meta[st].row;
+                    nvalid = meta[st].nvalid;
+                    pc = meta[st].piece;
+                }
+            }
+            if (row != cur_row || pc != cur_pc) {
+                if (cur_row >= 0) write_partial(cur_row, cur_pc);
+                if (row < 0) break;
+                start_row(row);
+                cur_row = row;
+                cur_pc = pc;
+            }
+
+            const uint32_t sK = stage0 + (uint32_t)st * STAGE_BYTES;
+            attend_tile<D, NT>(sK, sK + TILE_BYTES, nvalid, a.scale_log2, qf, acc, m_run, l_run, lane);
+            __syncwarp();  // every lane is done with this stage before it is refilled
+            ++consumed;
+        }
     }
 }
 
@@ -418,8 +524,9 @@ template <int D, int NT>
 static cudaError_t launch_gqa_dn(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                                  int grid, cudaStream_t s, bool pdl) {
     constexpr int STAGE_BYTES = 2 * DEC_TILE * D * 2;
-    const size_t smem = 1024 + (size_t)DEC_WARPS * DEC_STAGES * (STAGE_BYTES + 8 + sizeof(TileMeta));
     const bool late = a.chunks > a.static_chunks;
+    const size_t smem = 1024 + (size_t)DEC_WARPS * DEC_STAGES *
+                                   (STAGE_BYTES + 8 + (late ? sizeof(TileMeta<true>) : sizeof(TileMeta<false>)));
     auto kern = late ? k_decode_gqa<D, NT, true> : k_decode_gqa<D, NT, false>;
     static std::atomic<unsigned long long> done[2];
     cudaError_t e = ensure_smem_limit(kern, (int)smem, done[late ? 1 : 0]);

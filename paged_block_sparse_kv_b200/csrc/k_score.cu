@@ -160,14 +160,7 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
         pre_j = static_cast<int32_t>(p_begin + lane - prefix[pre_b]);
         pre_raw = a.page_indices[pptr[pre_b] + pre_j];
     }
-    if (a.table_ready) pdl_wait();
-    if (bad_len && blockIdx.x == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
-    // the decode kernel later in the same step counts its late pieces from this word
-    if (a.zero_word && blockIdx.x == 0 && threadIdx.x == 0) *a.zero_word = 0u;
-
-    // ---- group-summed queries of the block's first requests, computed once per block: each
-    // thread sums one (request, KV head, 8-dim chunk) over the group's heads in head order
-    float *qs = reinterpret_cast<float *>(smem + head_bytes + (size_t)SCORE_WARPS * per_warp_bytes);  // [qcap][Hkv][D]
+    // the block's first requests, whose group-summed queries it keeps in shared memory
     int qb0 = 0, qn = 0;
     {
         const int64_t bp0 = (int64_t)blockIdx.x * SCORE_WARPS * T / W;
@@ -176,6 +169,23 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32, 1) k_score_pages(ScoreArgs a
             qb0 = request_of(bp0);
             qn = min(a.qcap, request_of(bp1 - 1) - qb0 + 1);
         }
+    }
+    if (a.table_ready) {
+        // their query rows go to L2 while the previous kernel finishes (q itself is read only
+        // after the wait)
+        const char *q0 = reinterpret_cast<const char *>(a.q + (size_t)qb0 * a.Hq * D);
+        const int lines = static_cast<int>(((size_t)qn * a.Hq * D * 2 + 127) / 128);
+        for (int i = threadIdx.x; i < lines; i += blockDim.x) prefetch_l2(q0 + (size_t)i * 128);
+        pdl_wait();
+    }
+    if (bad_len && blockIdx.x == 0) set_err(a.err, VX_DATA_BAD_SEQ_LEN);
+    // the decode kernel later in the same step counts its late pieces from this word
+    if (a.zero_word && blockIdx.x == 0 && threadIdx.x == 0) *a.zero_word = 0u;
+
+    // ---- group-summed queries of the block's first requests, computed once per block: each
+    // thread sums one (request, KV head, 8-dim chunk) over the group's heads in head order
+    float *qs = reinterpret_cast<float *>(smem + head_bytes + (size_t)SCORE_WARPS * per_warp_bytes);  // [qcap][Hkv][D]
+    {
         constexpr int CPR = D / 8;  // 8-dim chunks per head row
         for (int idx = threadIdx.x; idx < qn * a.Hkv * CPR; idx += blockDim.x) {
             const int ch = idx % CPR, bh = idx / CPR;
