@@ -30,6 +30,9 @@ CASES = {
     # of them out late, in pieces, from a counter; short contexts leave -1 selection slots
     "late_pieces_b64": (synth.custom_spec(batch=64, num_q_heads=16, num_kv_heads=8, head_dim_qk=128, page_size=16,
                                           ctx=("uniform", 1500, 5000), k=160), 20),
+    # few rows of 1025..6144 pages: the 512-thread top-k blocks
+    "topk_rows_512": (synth.custom_spec(batch=2, num_q_heads=4, num_kv_heads=2, head_dim_qk=64, page_size=16,
+                                        ctx=("list", [20000, 70000]), k=100), 21),
     "mla_16heads": (synth.custom_spec(batch=3, num_q_heads=16, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
                                       page_size=64, mla_shared_kv=True, ctx=("list", [700, 2000, 64]), k=6), 17),
     "mla_5heads_ragged": (synth.custom_spec(batch=2, num_q_heads=5, num_kv_heads=1, head_dim_qk=576, head_dim_v=512,
@@ -142,7 +145,8 @@ def test_physical_page_permutation_is_bit_identical():
                            y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32))
 
 
-@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "g1_many_rows", "g16_d64_page64", "mla_16heads"])
+@pytest.mark.parametrize("name", ["qwen_shape_small_batch", "g1_many_rows", "g16_d64_page64", "mla_16heads",
+                                  "topk_rows_512"])
 def test_approx_topk_bit_exact_on_gpu_scores(name):
     w = workload(name)
     h = host(w)
