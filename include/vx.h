@@ -167,10 +167,12 @@ vx_status vx_topk_pages(const vx_geometry *geo, const vx_page_table *table, cons
  * distinct).  Split-K: the selected tokens are cut into contiguous chunks whose partial
  * (o, max, sum) are merged, in chunk order, with the log-sum-exp rule.
  *   num_splits > 0: that many chunks of equal length (in 16-token tiles; MLA: pages).
- *   num_splits 0: planned from the SM count.  MLA: one equal chunk per SM.  GQA: one equal
- *   chunk per warp of a persistent grid over the first three quarters of the tiles, then
- *   shorter equal chunks over the rest, each taken by whichever warp is free first.  The
- *   chunks are fixed before launch, so results never depend on timing.
+ *   num_splits 0: planned from the SM count.  MLA: the fewest equal chunks, at most one per
+ *   SM, that give no chunk more pages than one per SM would (128 for 512 pages on 148
+ *   SMs).  GQA: one equal chunk per warp of a persistent grid (8 warps per SM); when a
+ *   warp's share is 64 tiles or more, equal chunks per warp over the first three quarters
+ *   of the tiles, then shorter equal chunks over the rest, each taken by whichever warp is
+ *   free first.  The chunks are fixed before launch, so results never depend on timing.
  *   sm_scale <= 0 means 1 / sqrt(head_dim_qk).
  *   lse may be NULL.  A request with no attended token gets out = 0, lse = -inf.
  * ws: device workspace for the split partials; vx_workspace_size(geo, max_pages, k,
