@@ -50,8 +50,9 @@ DECODE_TRAFFIC = [
      "note": "captured at batch 160 (672.5 MB per launch, two steps; the split with late pieces, as at batch 256), "
              "scaled to the full launch by its bytes"},
     {"file": "csrc/k_decode_mla.cu", "sha256": "22e81ccb531f4f8aa2fb7013d797d94d058073446b7d6bf9de54dc1da54b31da",
-     "ratio": (38.158848 + 0.0576 + 38.157056 + 0.003072) / (2 * 38.264896), "workload": "mla_576_512_b16",
-     "note": "two consecutive launches of the full workload (2 input copies), 1-pass dram__bytes capture"},
+     "ratio": (38.15936 + 0.050944 + 38.155264 + 0.000256) / (2 * 38.264896), "workload": "mla_576_512_b16",
+     "note": "two consecutive launches of the full workload (2 input copies, the planned 128-CTA split), "
+             "1-pass dram__bytes capture"},
 ]
 
 

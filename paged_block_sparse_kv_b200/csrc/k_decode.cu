@@ -23,7 +23,8 @@
 // Per warp: a ring of DEC_STAGES stages in shared memory, each holding one K tile and
 // one V tile (16 tokens x D bf16 each), each filled by one TMA tensor load (128-byte
 // swizzle; a 4-D view lands the tile as D / 64 consecutive boxes of 16 rows x 64 columns)
-// that completes on a per-stage mbarrier.  Unit metadata (selected
+// that completes on a per-stage mbarrier.  A warp whose next tile has not landed sleeps in
+// mbarrier try_wait rather than spinning, so the SM's other warps get the issue slots.  Unit metadata (selected
 // page, physical page, valid tokens) is resolved 32 units at a time, one per lane.
 // Per tile: S^T = K Q^T with mma.m16n8k16 (tokens x heads, heads padded to 8 per
 // n-tile), online softmax in base 2, P^T moved into the B-operand layout with
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             int st = 0;
             if (!failed && consumed != issued) {
                 st = static_cast<int>(consumed % DEC_STAGES);
-                if (!__all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
+                if (!__all_sync(FULL, mbar_wait_sleep(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
                     // a load did not arrive in time: report, let every issued load land and
                     // finish the remaining rows as empty
                     if (lane == 0) set_err(a.err, VX_DATA_TIMEOUT);
@@ -383,7 +384,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             int st = 0;
             if (!failed && consumed != issued) {
                 st = static_cast<int>(consumed % DEC_STAGES);
-                if (!__all_sync(FULL, mbar_wait_bounded(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
+                if (!__all_sync(FULL, mbar_wait_sleep(bar0 + 8u * st, (consumed / DEC_STAGES) & 1u))) {
                     // a load did not arrive in time: report, let every issued load land, drop the
                     // partial in progress (its slot keeps its empty partial) and give every piece
                     // this warp would still have taken its empty partials

@@ -116,6 +116,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, unsigned parity)
     }
 }
 
+// Like mbar_wait_bounded, but a waiter that misses the first test sleeps in try_wait with a
+// suspend hint instead of spinning, leaving the issue slots to the warps doing math.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, unsigned parity) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
+        if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
+    }
+}
+
 // ------------------------------------------------------------------- TMA
 
 // 3-D tiled tensor load global -> shared, completion counted on `bar` in bytes.
