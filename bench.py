@@ -39,14 +39,14 @@ DEFAULT_CONFIG = "qwen3_1p7b_gqa_b32"
 # as a multiple of the algorithmic bytes of the captured launch, per (kernel source, workload); valid only
 # for the kernel source it was taken on (sha256 of the file), otherwise the bench reports null.
 DECODE_TRAFFIC = [
-    {"file": "csrc/k_decode.cu", "sha256": "3a253af780bb7ce71e165fefbf35c3d8e7b936d7ed56034becf5360cf92eb611",
-     "ratio": (268.90496 + 3.272192 + 268.929536 + 0.264448) / (2 * 268.511488), "workload": "qwen3_1p7b_gqa_b32",
+    {"file": "csrc/k_decode.cu", "sha256": "836824bf1089964ce4de52184d5e180253562ffb75dbade3387bb195cbaeab2f",
+     "ratio": (268.934912 + 3.29856 + 268.955392 + 0.409856) / (2 * 268.511488), "workload": "qwen3_1p7b_gqa_b32",
      "note": "two consecutive launches of the full workload (2 input copies), 1-pass dram__bytes capture"},
-    {"file": "csrc/k_decode.cu", "sha256": "3a253af780bb7ce71e165fefbf35c3d8e7b936d7ed56034becf5360cf92eb611",
-     "ratio": (67.367168 + 0.921856 + 67.364864 + 0.086784) / (2 * 67.1744), "workload": "long_ctx_128k_b8",
+    {"file": "csrc/k_decode.cu", "sha256": "836824bf1089964ce4de52184d5e180253562ffb75dbade3387bb195cbaeab2f",
+     "ratio": (67.366656 + 0.883456 + 67.365888 + 0.361984) / (2 * 67.1744), "workload": "long_ctx_128k_b8",
      "note": "captured at batch 4 (67.2 MB per launch, two launches), scaled to the full launch by its bytes"},
-    {"file": "csrc/k_decode.cu", "sha256": "3a253af780bb7ce71e165fefbf35c3d8e7b936d7ed56034becf5360cf92eb611",
-     "ratio": (674.102784 + 8.412416 + 674.006784 + 5.035264) / (2 * 672.470302), "workload": "cont_batch_b256",
+    {"file": "csrc/k_decode.cu", "sha256": "836824bf1089964ce4de52184d5e180253562ffb75dbade3387bb195cbaeab2f",
+     "ratio": (674.105088 + 8.291072 + 674.06336 + 5.162496) / (2 * 672.470302), "workload": "cont_batch_b256",
      "note": "captured at batch 160 (672.5 MB per launch, two steps; the split with late pieces, as at batch 256), "
              "scaled to the full launch by its bytes"},
     {"file": "csrc/k_decode_mla.cu", "sha256": "22e81ccb531f4f8aa2fb7013d797d94d058073446b7d6bf9de54dc1da54b31da",

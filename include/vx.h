@@ -185,16 +185,6 @@ vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, c
                            size_t ws_bytes, int32_t *err, void *stream);
 
 /*
- * One whole decode step: vx_score_pages -> vx_topk_pages -> vx_sparse_decode, chained
- * on `stream` with programmatic dependent launch so each kernel's start overlaps the
- * previous one's tail (paper note, 系统设计 3: fusion of the sequence-local steps and
- * workload planning).  Same arguments and results as the three calls.  scores_out and
- * sel_out (may be NULL) receive the intermediate scores and selection; when NULL they
- * live in the workspace.  score_dims as in vx_score_pages.  ws: vx_workspace_size bytes,
- * no initial contents needed.
- * mode: vx_topk_pages's mode (0..3), optionally OR-ed with VX_TABLE_READY.
- */
-/*
  * Flag OR-ed into the mode of the two chained steps below.  It promises that the page table
  * (page_ptr, page_indices) and seq_lens were not written by the last kernel launched on the
  * stream before the call (they came from host copies, or from an earlier kernel).  The
@@ -206,6 +196,16 @@ vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, c
  */
 #define VX_TABLE_READY 0x100
 
+/*
+ * One whole decode step: vx_score_pages -> vx_topk_pages -> vx_sparse_decode, chained
+ * on `stream` with programmatic dependent launch so each kernel's start overlaps the
+ * previous one's tail (paper note, 系统设计 3: fusion of the sequence-local steps and
+ * workload planning).  Same arguments and results as the three calls.  scores_out and
+ * sel_out (may be NULL) receive the intermediate scores and selection; when NULL they
+ * live in the workspace.  score_dims as in vx_score_pages.  ws: vx_workspace_size bytes,
+ * no initial contents needed.
+ * mode: vx_topk_pages's mode (0..3), optionally OR-ed with VX_TABLE_READY.
+ */
 vx_status vx_block_topk_decode(const vx_geometry *geo, const vx_page_table *table, const void *q,
                                const void *k_cache, const void *v_cache, const void *centroids,
                                int32_t k, int32_t mode, uint64_t seed, float sm_scale,
