@@ -177,7 +177,9 @@ vx_status vx_topk_pages(const vx_geometry *geo, const vx_page_table *table, cons
  *   lse may be NULL.  A request with no attended token gets out = 0, lse = -inf.
  * ws: device workspace for the split partials; vx_workspace_size(geo, max_pages, k,
  * num_splits) bytes are always enough (that size also covers the fused call's scores
- * and selection, which this call does not use).
+ * and selection, which this call does not use).  No initial contents needed: when the
+ * planned split has late chunks, the call first zeroes their counter, one word of ws, with
+ * a 4-byte cudaMemsetAsync on `stream`.
  */
 vx_status vx_sparse_decode(const vx_geometry *geo, const vx_page_table *table, const void *q,
                            const void *k_cache, const void *v_cache, const int32_t *sel, int32_t k,
